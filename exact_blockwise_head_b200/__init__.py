@@ -1,0 +1,184 @@
+"""Exact blockwise multi-head attention forward for B200 (sm_100a).
+
+A thin Python binding over the C ABI of ``include/attn.h`` (libebh_attn.so).
+This module only marshals arguments -- every step of the attention runs in
+the library's CUDA kernels.  PyTorch provides device memory and streams.
+
+    >>> from exact_blockwise_head_b200 import forward
+    >>> out, lse = forward(q, k, v, mask="causal")      # q, k, v: [B, H, L, d]
+
+There is no CPU fallback: if the library is missing or the device is not a
+B200, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+from .workloads import MASK_KINDS, WORKLOADS, Workload, make_qkv, sample_rows  # noqa: F401
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libebh_attn.so")
+
+ATTN_OK = 0
+ATTN_ERR_INVALID = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_MISALIGNED = 3
+ATTN_ERR_CUDA = 4
+ATTN_ERR_TIMEOUT = 5
+ATTN_DTYPE_BF16 = 0
+ATTN_DTYPE_F32 = 1
+
+# Every entry point declared in include/attn.h.
+EXPORTED = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ex", "attn_strerror", "attn_last_cuda_error",
+            "attn_device_status", "attn_selftest_wait_timeout", "attn_kv_tile_range",
+            "attn_kv_tile_class", "attn_abi_version")
+
+
+class AttnParams(ctypes.Structure):
+    """Mirror of ``attn_params`` in include/attn.h."""
+    _fields_ = [
+        ("dtype", ctypes.c_int),
+        ("q", ctypes.c_void_p),
+        ("k", ctypes.c_void_p),
+        ("v", ctypes.c_void_p),
+        ("out", ctypes.c_void_p),
+        ("lse", ctypes.c_void_p),
+        ("B", ctypes.c_int),
+        ("H", ctypes.c_int),
+        ("L", ctypes.c_int),
+        ("d", ctypes.c_int),
+        ("scale", ctypes.c_float),
+        ("mask_kind", ctypes.c_int),
+        ("window", ctypes.c_int),
+        ("block_n", ctypes.c_int),
+        ("wait_timeout_ns", ctypes.c_uint64),
+    ]
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = _load()
+        msg = lib.attn_strerror(status).decode()
+        if status == ATTN_ERR_CUDA:
+            msg += f" (cudaError {lib.attn_last_cuda_error()})"
+        super().__init__(f"{where}: {msg}")
+        self.status = status
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def _load():
+    """Load libebh_attn.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"{LIB_PATH} is missing: build it with "
+                                  "`python -m exact_blockwise_head_b200.build`")
+            lib = ctypes.CDLL(LIB_PATH)
+            vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+            lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+            lib.attn_fwd_f32.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, vp]
+            lib.attn_fwd_ex.argtypes = [ctypes.POINTER(AttnParams), vp]
+            lib.attn_strerror.argtypes = [i]
+            lib.attn_strerror.restype = ctypes.c_char_p
+            lib.attn_last_cuda_error.argtypes = []
+            lib.attn_device_status.argtypes = [i, i]
+            lib.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+            lib.attn_kv_tile_range.argtypes = [i, i, i, i, i, i, ctypes.POINTER(i),
+                                               ctypes.POINTER(i)]
+            lib.attn_kv_tile_class.argtypes = [i, i, i, i, i, i, i]
+            lib.attn_abi_version.argtypes = []
+            for name in EXPORTED:
+                if name != "attn_strerror":
+                    getattr(lib, name).restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def library():
+    """The loaded ctypes library (for tests and tools that call the ABI directly)."""
+    return _load()
+
+
+def _stream_handle(stream, device):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def forward(q, k, v, scale=None, mask="none", window=0, block_n=0, out=None, lse=None,
+            want_lse=True, stream=None, wait_timeout_ns=0):
+    """O = softmax(scale * Q K^T + mask) V and the per-row log-sum-exp.
+
+    q, k, v: CUDA tensors of one shape [B, H, L, d], all bf16 (tensor-core path,
+    d in {64, 128}) or all fp32 (CUDA-core path, d <= 256), contiguous.
+    mask: "none", "causal" (key j <= query i) or "window" (|i - j| <= window).
+    scale defaults to 1/sqrt(d).  Returns (out, lse); lse is None when
+    want_lse is False.  The work is enqueued on `stream` (default: the current
+    stream) and the call returns without synchronising.
+    """
+    import torch
+
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("q, k, v must be bf16 or fp32")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share one [B, H, L, d] shape")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    B, H, L, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if mask not in MASK_KINDS:
+        raise ValueError(f"mask must be one of {sorted(MASK_KINDS)}")
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    p = AttnParams()
+    p.dtype = ATTN_DTYPE_BF16 if q.dtype == torch.bfloat16 else ATTN_DTYPE_F32
+    p.q, p.k, p.v, p.out = q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr()
+    p.lse = lse.data_ptr() if (want_lse and lse is not None) else None
+    p.B, p.H, p.L, p.d = B, H, L, d
+    p.scale = float(scale)
+    p.mask_kind = MASK_KINDS[mask]
+    p.window = int(window)
+    p.block_n = int(block_n)
+    p.wait_timeout_ns = int(wait_timeout_ns)
+    with torch.cuda.device(q.device):
+        st = _load().attn_fwd_ex(ctypes.byref(p), _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_ex")
+    return out, (lse if want_lse else None)
+
+
+def device_status(device: int = 0, reset: bool = True) -> int:
+    """Read (and clear) the per-device status word that kernels set when a
+    bounded wait runs out.  Synchronises with the device."""
+    return _load().attn_device_status(int(device), 1 if reset else 0)
+
+
+def kv_tile_range(L, q_first, q_last, mask="none", window=0, block_n=128):
+    lo, hi = ctypes.c_int(), ctypes.c_int()
+    st = _load().attn_kv_tile_range(L, q_first, q_last, MASK_KINDS[mask], window, block_n,
+                                    ctypes.byref(lo), ctypes.byref(hi))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_kv_tile_range")
+    return lo.value, hi.value
+
+
+def kv_tile_class(L, q_first, q_last, j, mask="none", window=0, block_n=128):
+    c = _load().attn_kv_tile_class(L, q_first, q_last, j, MASK_KINDS[mask], window, block_n)
+    if c < 0:
+        raise AttnError(-c, "attn_kv_tile_class")
+    return c

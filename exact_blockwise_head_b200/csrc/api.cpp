@@ -1,0 +1,220 @@
+// api.cpp -- the C ABI declared in include/attn.h: argument validation, path
+// selection and the host copies of the tile rule.  Every check runs before
+// anything is launched; nothing here allocates device memory or synchronises
+// (except attn_device_status, which is documented to).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "kernels.h"
+#include "tiles.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+constexpr uint64_t kDefaultTimeoutNs = 10ull * 1000 * 1000 * 1000;
+
+int fail_cuda(cudaError_t e) {
+  g_last_cuda_error = static_cast<int>(e);
+  return ATTN_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Half-open byte ranges [a, a + na) and [b, b + nb) overlap?
+bool overlap(const void* a, uint64_t na, const void* b, uint64_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// Validation common to both paths; fills `out` with the normalised problem.
+int validate(const attn_params* p, ebh::FwdArgs* out) {
+  if (p == nullptr) return ATTN_ERR_INVALID;
+  if (p->dtype != ATTN_DTYPE_BF16 && p->dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID;
+  if (!p->q || !p->k || !p->v || !p->out) return ATTN_ERR_INVALID;
+  if (p->B <= 0 || p->H <= 0 || p->L <= 0 || p->d <= 0) return ATTN_ERR_INVALID;
+  if (static_cast<long long>(p->B) * p->H > 0x7fffffffLL) return ATTN_ERR_INVALID;
+  if (!std::isfinite(p->scale) || !(p->scale > 0.f)) return ATTN_ERR_INVALID;
+  if (p->mask_kind != ATTN_MASK_NONE && p->mask_kind != ATTN_MASK_CAUSAL &&
+      p->mask_kind != ATTN_MASK_WINDOW)
+    return ATTN_ERR_INVALID;
+  if (p->mask_kind == ATTN_MASK_WINDOW && p->window < 0) return ATTN_ERR_INVALID;
+  if (p->dtype == ATTN_DTYPE_BF16) {
+    if (p->block_n != 0 && p->block_n != 64 && p->block_n != 128) return ATTN_ERR_INVALID;
+  } else if (p->block_n != 0) {
+    return ATTN_ERR_INVALID;
+  }
+  const uint64_t elem = p->dtype == ATTN_DTYPE_BF16 ? 2 : 4;
+  const uint64_t rows = static_cast<uint64_t>(p->B) * p->H * p->L;
+  const uint64_t tensor_bytes = rows * p->d * elem;
+  const uint64_t lse_bytes = rows * 4;
+  if (overlap(p->out, tensor_bytes, p->q, tensor_bytes) ||
+      overlap(p->out, tensor_bytes, p->k, tensor_bytes) ||
+      overlap(p->out, tensor_bytes, p->v, tensor_bytes))
+    return ATTN_ERR_INVALID;
+  if (p->lse && (overlap(p->lse, lse_bytes, p->q, tensor_bytes) ||
+                 overlap(p->lse, lse_bytes, p->k, tensor_bytes) ||
+                 overlap(p->lse, lse_bytes, p->v, tensor_bytes) ||
+                 overlap(p->lse, lse_bytes, p->out, tensor_bytes)))
+    return ATTN_ERR_INVALID;
+  if (p->dtype == ATTN_DTYPE_BF16) {
+    if (p->d != 64 && p->d != 128) return ATTN_ERR_UNSUPPORTED;
+  } else if (p->d > 256) {
+    return ATTN_ERR_UNSUPPORTED;
+  }
+  if (!aligned(p->q, 16) || !aligned(p->k, 16) || !aligned(p->v, 16) || !aligned(p->out, 16))
+    return ATTN_ERR_MISALIGNED;
+  if (p->lse && !aligned(p->lse, 4)) return ATTN_ERR_MISALIGNED;
+
+  out->q = p->q;
+  out->k = p->k;
+  out->v = p->v;
+  out->out = p->out;
+  out->lse = p->lse;
+  out->B = p->B;
+  out->H = p->H;
+  out->L = p->L;
+  out->d = p->d;
+  out->scale = p->scale;
+  out->mask_kind = p->mask_kind;
+  // a band at least L wide allows every pair: clamp so index sums stay small
+  out->window = p->mask_kind == ATTN_MASK_WINDOW ? (p->window > p->L ? p->L : p->window) : 0;
+  out->block_n = p->dtype == ATTN_DTYPE_BF16 ? (p->block_n == 0 ? 128 : p->block_n) : 0;
+  out->timeout_ns = p->wait_timeout_ns ? p->wait_timeout_ns : kDefaultTimeoutNs;
+  return ATTN_OK;
+}
+
+// The tensor-core path needs a compute-capability 10.0 device (sm_100a code).
+int check_device_sm100() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e);
+  static std::mutex mu;
+  static int cc[64] = {0};
+  std::lock_guard<std::mutex> g(mu);
+  if (dev < 0 || dev >= 64) return fail_cuda(cudaErrorInvalidDevice);
+  if (cc[dev] == 0) {
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) !=
+        cudaSuccess)
+      return fail_cuda(e);
+    if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) !=
+        cudaSuccess)
+      return fail_cuda(e);
+    cc[dev] = major * 10 + minor;
+  }
+  return cc[dev] == 100 ? ATTN_OK : ATTN_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd_ex(const attn_params* p, void* stream) {
+  ebh::FwdArgs a;
+  int st = validate(p, &a);
+  if (st != ATTN_OK) return st;
+  if ((st = check_device_sm100()) != ATTN_OK) return st;
+  cudaError_t err = cudaSuccess;
+  st = p->dtype == ATTN_DTYPE_BF16
+           ? ebh::launch_fwd_bf16_sm100(a, static_cast<cudaStream_t>(stream), &err)
+           : ebh::launch_fwd_f32(a, static_cast<cudaStream_t>(stream), &err);
+  if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
+  return st;
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
+             int L, int d, float scale, int mask_kind, int window, void* stream) {
+  attn_params p = {};
+  p.dtype = ATTN_DTYPE_BF16;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.out = out;
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.L = L;
+  p.d = d;
+  p.scale = scale;
+  p.mask_kind = mask_kind;
+  p.window = window;
+  return attn_fwd_ex(&p, stream);
+}
+
+int attn_fwd_f32(const float* q, const float* k, const float* v, float* out, float* lse, int B,
+                 int H, int L, int d, float scale, int mask_kind, int window, void* stream) {
+  attn_params p = {};
+  p.dtype = ATTN_DTYPE_F32;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.out = out;
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.L = L;
+  p.d = d;
+  p.scale = scale;
+  p.mask_kind = mask_kind;
+  p.window = window;
+  return attn_fwd_ex(&p, stream);
+}
+
+const char* attn_strerror(int status) {
+  switch (status) {
+    case ATTN_OK: return "success";
+    case ATTN_ERR_INVALID: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported head dimension, size or device";
+    case ATTN_ERR_MISALIGNED: return "misaligned pointer (q/k/v/out need 16 bytes, lse 4)";
+    case ATTN_ERR_CUDA: return "CUDA runtime error (see attn_last_cuda_error)";
+    case ATTN_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    default: return "unknown status";
+  }
+}
+
+int attn_last_cuda_error(void) { return g_last_cuda_error; }
+
+int attn_device_status(int device, int reset) {
+  cudaError_t err = cudaSuccess;
+  int st = ebh::read_device_status(device, reset, &err);
+  if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
+  return st;
+}
+
+int attn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns == 0) return ATTN_ERR_INVALID;
+  int st = check_device_sm100();
+  if (st != ATTN_OK) return st;
+  cudaError_t err = cudaSuccess;
+  st = ebh::launch_selftest_wait_timeout(limit_ns, static_cast<cudaStream_t>(stream), &err);
+  if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
+  return st;
+}
+
+int attn_kv_tile_range(int L, int q_first, int q_last, int mask_kind, int window, int block_n,
+                       int* lo, int* hi) {
+  if (!lo || !hi || L <= 0 || block_n <= 0 || q_first < 0 || q_last < q_first || q_last >= L)
+    return ATTN_ERR_INVALID;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_WINDOW) return ATTN_ERR_INVALID;
+  if (mask_kind == ATTN_MASK_WINDOW && window < 0) return ATTN_ERR_INVALID;
+  ebh::kv_tile_range(L, q_first, q_last, mask_kind, window, block_n, *lo, *hi);
+  return ATTN_OK;
+}
+
+int attn_kv_tile_class(int L, int q_first, int q_last, int j, int mask_kind, int window,
+                       int block_n) {
+  if (L <= 0 || block_n <= 0 || q_first < 0 || q_last < q_first || q_last >= L)
+    return -ATTN_ERR_INVALID;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_WINDOW) return -ATTN_ERR_INVALID;
+  if (mask_kind == ATTN_MASK_WINDOW && window < 0) return -ATTN_ERR_INVALID;
+  return ebh::kv_tile_class(L, q_first, q_last, j, mask_kind, window, block_n);
+}
+
+int attn_abi_version(void) { return ATTN_ABI_VERSION; }
+
+}  // extern "C"

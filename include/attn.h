@@ -1,0 +1,172 @@
+/*
+ * attn.h -- C ABI of the exact blockwise multi-head attention forward
+ * (libebh_attn.so).
+ *
+ * Operation.  For every batch b, head h and query row i:
+ *     O[b,h,i,:] = sum_j softmax_j( scale * <Q[b,h,i,:], K[b,h,j,:]> + mask(i,j) ) V[b,h,j,:]
+ *     LSE[b,h,i] = ln sum_{j allowed} exp( scale * <Q[b,h,i,:], K[b,h,j,:]> )
+ * the formula softmax(Q K^T / sqrt(d_k)) V of the page "Transformer multi-head
+ * attention, 8-head parallel computation: PyTorch implementation and CUDA
+ * kernel optimisation" (lshu.cn), section 1, with the scores of disallowed keys
+ * set to -inf before the softmax as in its section 2.2.  The result is exact
+ * up to rounding: it is computed tile by tile over blocks of keys with a
+ * running max and sum (the fused kernel of the page "Mosaic multi-GPU
+ * sequence-sharded attention" (kwkr.cn), section 3.2, with the rescale that
+ * sketch omits), so the L x L score matrix is never stored and memory stays
+ * O(L), as the query-blockwise scheme of "Blockwise Parallel Transformer in
+ * PyTorch" (qqiyuan.cn) intends.
+ *
+ * Masks.
+ *   ATTN_MASK_NONE    every key j in [0, L)
+ *   ATTN_MASK_CAUSAL  j <= i (diagonal included; queries and keys aligned)
+ *   ATTN_MASK_WINDOW  |i - j| <= window, the band of "Attention optimisation
+ *                     strategies and practice for long-sequence inference"
+ *                     (trdm.cn), section 2.1, applied additively (-inf)
+ * Every mask allows the diagonal, so no row is ever fully masked.
+ *
+ * Layout.  q, k, v, out are dense row-major [B, H, L, d] arrays (d fastest,
+ * then L, then H, then B) in device memory.  lse is a dense [B, H, L] fp32
+ * array in device memory, or NULL to skip it.
+ *
+ * Ownership and execution.  The caller owns every buffer.  Each call only
+ * enqueues work on `stream` (a cudaStream_t; NULL = the legacy default
+ * stream) and returns: it never allocates or frees device memory and never
+ * synchronises.  The buffers must stay valid until the work completes.  `out`
+ * and `lse` must not overlap q, k, v or each other.  Calls are thread-safe.
+ *
+ * Errors.  Every argument is validated before anything is launched; a call
+ * that returns an error has enqueued nothing (except ATTN_ERR_CUDA, which
+ * reports a failed launch).  attn_strerror() names a status.  Waits inside
+ * the kernels are bounded: if one runs out (a malfunction, never expected),
+ * the kernel records ATTN_ERR_TIMEOUT in a per-device status word, releases
+ * its resources and returns; attn_device_status() reads that word.
+ */
+#ifndef EBH_ATTN_H
+#define EBH_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ATTN_ABI_VERSION 1
+
+/* Symbol visibility: the library is built with hidden visibility by default
+ * and exports exactly the entry points declared here. */
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+/* Status codes returned by every entry point. */
+enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID = 1,     /* null pointer, non-positive size, bad mask kind,
+                               negative window, non-finite or non-positive
+                               scale, overlapping outputs, bad block_n/dtype */
+  ATTN_ERR_UNSUPPORTED = 2, /* head dim not supported by the chosen path, or
+                               the current device is not sm_100 */
+  ATTN_ERR_MISALIGNED = 3,  /* q/k/v/out not 16-byte aligned, lse not 4-byte */
+  ATTN_ERR_CUDA = 4,        /* a CUDA runtime call failed; attn_last_cuda_error()
+                               gives its code */
+  ATTN_ERR_TIMEOUT = 5      /* a bounded wait inside a kernel ran out */
+};
+
+/* Mask kinds. */
+enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1, ATTN_MASK_WINDOW = 2 };
+
+/* Element types. */
+enum { ATTN_DTYPE_BF16 = 0, ATTN_DTYPE_F32 = 1 };
+
+/* Tile classes returned by attn_kv_tile_class(). */
+enum { ATTN_TILE_EMPTY = 0, ATTN_TILE_PARTIAL = 1, ATTN_TILE_FULL = 2 };
+
+/*
+ * bf16 forward on the sm_100a tensor cores (tcgen05 MMAs into tensor memory,
+ * TMA-staged tiles).  q, k, v, out: bf16 [B,H,L,d], d in {64, 128}, 16-byte
+ * aligned.  lse: fp32 [B,H,L] or NULL.  Products accumulate in fp32; the
+ * softmax runs in fp32 with exp2; the probabilities are rounded to bf16 for
+ * the P.V product; out is rounded to bf16 (nearest-even).  B, H, L >= 1 with
+ * B*H <= 2^31-1; scale finite and > 0 (the pages use 1/sqrt(d)); window >= 0,
+ * read only for ATTN_MASK_WINDOW.  Keys are visited in blocks of 128.
+ */
+ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+             int B, int H, int L, int d, float scale, int mask_kind, int window,
+             void* stream);
+
+/*
+ * fp32 forward on the CUDA cores (exact fp32 arithmetic, expf): q, k, v, out
+ * fp32 [B,H,L,d] with 1 <= d <= 256, 16-byte aligned; other arguments as for
+ * attn_fwd.  This path keeps full fp32 precision (no TF32).
+ */
+ATTN_API int attn_fwd_f32(const float* q, const float* k, const float* v, float* out,
+                 float* lse, int B, int H, int L, int d, float scale,
+                 int mask_kind, int window, void* stream);
+
+/* Full parameter set for attn_fwd_ex(). */
+typedef struct attn_params {
+  int dtype;              /* ATTN_DTYPE_BF16 or ATTN_DTYPE_F32 */
+  const void* q;          /* [B,H,L,d] */
+  const void* k;          /* [B,H,L,d] */
+  const void* v;          /* [B,H,L,d] */
+  void* out;              /* [B,H,L,d], same dtype as q */
+  float* lse;             /* [B,H,L] fp32, or NULL */
+  int B, H, L, d;
+  float scale;
+  int mask_kind;
+  int window;
+  int block_n;            /* keys per block on the bf16 path: 0 (auto = 128),
+                             64 or 128; must be 0 on the fp32 path */
+  uint64_t wait_timeout_ns; /* limit on each wait inside the kernel; 0 = 10 s */
+} attn_params;
+
+/* attn_fwd / attn_fwd_f32 with every knob exposed. */
+ATTN_API int attn_fwd_ex(const attn_params* p, void* stream);
+
+/* Static text for a status code (never NULL). */
+ATTN_API const char* attn_strerror(int status);
+
+/* The cudaError_t of the last ATTN_ERR_CUDA returned on this thread (0 if none). */
+ATTN_API int attn_last_cuda_error(void);
+
+/*
+ * Reads, and if `reset` clears, the status word that kernels on `device` set
+ * when a bounded wait ran out.  Returns ATTN_OK, ATTN_ERR_TIMEOUT, or
+ * ATTN_ERR_CUDA if the device could not be queried.  Unlike every other entry
+ * point this one synchronises with the device (it copies the word back).
+ */
+ATTN_API int attn_device_status(int device, int reset);
+
+/*
+ * Failure-detection self test: launches one CTA that waits on a barrier which
+ * nothing ever arrives on, with the limit `limit_ns`; the wait runs out, the
+ * kernel records ATTN_ERR_TIMEOUT in the device status word and returns
+ * normally.  Used to test the bounded-wait path without hanging a GPU.
+ */
+ATTN_API int attn_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+/*
+ * Host copies of the tile-skipping rule the kernels use.  Query rows
+ * [q_first, q_last] (inclusive, q_last < L) meet key blocks of block_n keys;
+ * attn_kv_tile_range() gives the half-open range [lo, hi) of key blocks that
+ * hold at least one allowed key, and attn_kv_tile_class() classifies block j
+ * as EMPTY (no allowed pair), PARTIAL (some pair masked, or keys past L) or
+ * FULL (every pair allowed).  attn_kv_tile_range returns ATTN_ERR_INVALID on
+ * bad arguments; attn_kv_tile_class returns -ATTN_ERR_INVALID (negative, so
+ * it cannot be mistaken for a class).
+ */
+ATTN_API int attn_kv_tile_range(int L, int q_first, int q_last, int mask_kind, int window,
+                       int block_n, int* lo, int* hi);
+ATTN_API int attn_kv_tile_class(int L, int q_first, int q_last, int j, int mask_kind,
+                       int window, int block_n);
+
+/* ATTN_ABI_VERSION of the loaded library. */
+ATTN_API int attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EBH_ATTN_H */

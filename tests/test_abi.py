@@ -1,0 +1,127 @@
+"""The C ABI loads, exports every declared entry point, and rejects bad
+arguments on the host before touching a GPU (CPU only: no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_blockwise_head_b200 as ebh
+from exact_blockwise_head_b200 import build as ebh_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ebh_build.build()
+    return ebh.library()
+
+
+def test_header_declares_the_python_list():
+    assert declared_symbols() == sorted(ebh.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    # nothing beyond the ABI leaks out of the library
+    out = os.popen(f"nm -D --defined-only {ebh.LIB_PATH}").read()
+    exported = sorted(l.split()[-1] for l in out.splitlines() if " T " in l)
+    assert exported == declared_symbols()
+
+
+def test_abi_version_and_strerror(lib):
+    assert lib.attn_abi_version() == 1
+    for code in range(0, 6):
+        assert lib.attn_strerror(code)
+    assert b"unknown" in lib.attn_strerror(99)
+
+
+def _params(**kw):
+    p = ebh.AttnParams()
+    p.dtype = kw.get("dtype", ebh.ATTN_DTYPE_BF16)
+    base = 1 << 20
+    size = 1 << 24
+    p.q = kw.get("q", base)
+    p.k = kw.get("k", base + size)
+    p.v = kw.get("v", base + 2 * size)
+    p.out = kw.get("out", base + 3 * size)
+    p.lse = kw.get("lse", base + 4 * size)
+    p.B, p.H, p.L, p.d = kw.get("B", 1), kw.get("H", 2), kw.get("L", 256), kw.get("d", 64)
+    p.scale = kw.get("scale", 0.125)
+    p.mask_kind = kw.get("mask_kind", 0)
+    p.window = kw.get("window", 0)
+    p.block_n = kw.get("block_n", 0)
+    p.wait_timeout_ns = 0
+    return p
+
+
+BAD = [
+    ("null q", dict(q=0), ebh.ATTN_ERR_INVALID),
+    ("null out", dict(out=0), ebh.ATTN_ERR_INVALID),
+    ("B=0", dict(B=0), ebh.ATTN_ERR_INVALID),
+    ("H<0", dict(H=-1), ebh.ATTN_ERR_INVALID),
+    ("L=0", dict(L=0), ebh.ATTN_ERR_INVALID),
+    ("d=0", dict(d=0), ebh.ATTN_ERR_INVALID),
+    ("scale nan", dict(scale=float("nan")), ebh.ATTN_ERR_INVALID),
+    ("scale inf", dict(scale=float("inf")), ebh.ATTN_ERR_INVALID),
+    ("scale 0", dict(scale=0.0), ebh.ATTN_ERR_INVALID),
+    ("scale<0", dict(scale=-1.0), ebh.ATTN_ERR_INVALID),
+    ("mask 3", dict(mask_kind=3), ebh.ATTN_ERR_INVALID),
+    ("mask -1", dict(mask_kind=-1), ebh.ATTN_ERR_INVALID),
+    ("window<0", dict(mask_kind=2, window=-1), ebh.ATTN_ERR_INVALID),
+    ("block_n 96", dict(block_n=96), ebh.ATTN_ERR_INVALID),
+    ("block_n 256", dict(block_n=256), ebh.ATTN_ERR_INVALID),
+    ("f32 block_n", dict(dtype=1, block_n=64), ebh.ATTN_ERR_INVALID),
+    ("dtype 7", dict(dtype=7), ebh.ATTN_ERR_INVALID),
+    ("out aliases q", dict(out=1 << 20), ebh.ATTN_ERR_INVALID),
+    ("out overlaps v", dict(out=(1 << 20) + 2 * (1 << 24) + 64), ebh.ATTN_ERR_INVALID),
+    ("lse inside out", dict(lse=(1 << 20) + 3 * (1 << 24) + 16), ebh.ATTN_ERR_INVALID),
+    ("bf16 d=96", dict(d=96), ebh.ATTN_ERR_UNSUPPORTED),
+    ("bf16 d=256", dict(d=256), ebh.ATTN_ERR_UNSUPPORTED),
+    ("f32 d=257", dict(dtype=1, d=257), ebh.ATTN_ERR_UNSUPPORTED),
+    ("q misaligned", dict(q=(1 << 20) + 8), ebh.ATTN_ERR_MISALIGNED),
+    ("out misaligned", dict(out=(1 << 20) + 3 * (1 << 24) + 2), ebh.ATTN_ERR_MISALIGNED),
+    ("lse misaligned", dict(lse=(1 << 20) + 4 * (1 << 24) + 2), ebh.ATTN_ERR_MISALIGNED),
+]
+
+
+@pytest.mark.parametrize("what,kw,code", BAD, ids=[b[0] for b in BAD])
+def test_bad_arguments_are_rejected_before_launch(lib, what, kw, code):
+    p = _params(**kw)
+    assert lib.attn_fwd_ex(ctypes.byref(p), None) == code
+
+
+def test_null_params(lib):
+    assert lib.attn_fwd_ex(None, None) == ebh.ATTN_ERR_INVALID
+
+
+def test_plain_entry_points_validate(lib):
+    assert lib.attn_fwd(0, 0, 0, 0, 0, 1, 1, 16, 64, 0.125, 0, 0, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_fwd_f32(0, 0, 0, 0, 0, 1, 1, 16, 64, 0.125, 0, 0, None) == \
+        ebh.ATTN_ERR_INVALID
+    assert lib.attn_selftest_wait_timeout(0, None) == ebh.ATTN_ERR_INVALID
+
+
+def test_valid_call_without_a_b200_does_not_launch(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; covered by the gpu tests")
+    p = _params()
+    st = lib.attn_fwd_ex(ctypes.byref(p), None)
+    assert st in (ebh.ATTN_ERR_CUDA, ebh.ATTN_ERR_UNSUPPORTED)
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """The binding has no CPU fallback: without the .so it raises."""
+    monkeypatch.setattr(ebh, "_lib", None)
+    monkeypatch.setattr(ebh, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(ImportError):
+        ebh.library()

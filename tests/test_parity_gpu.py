@@ -1,0 +1,136 @@
+"""Parity of the CUDA path (called through the C ABI) with the fp64 oracle.
+
+Small and ragged problems are compared element by element on every row; the
+five full-size workloads are compared on sampled rows (tile edges, the last
+rows, 56 random rows per head).  Tolerances: bf16 max |O-O*| <= 2e-2 and
+max |LSE-LSE*| <= 1e-3; fp32 1e-4 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+import exact_blockwise_head_b200 as ebh
+from tests import gpu_helpers as G
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    G.require_gpu()
+
+
+# ---------------------------------------------------------------- fp32 path
+def test_fp32_tiny_exact_attention():
+    """B=1, H=2, L=256, d=64, no mask, scale 1/8, N(0,1) from seed 0."""
+    w = ebh.WORKLOADS["tiny_f32_L256_d64"]
+    q, k, v = ebh.make_qkv(w)
+    out, lse = G.gpu_forward(q, k, v)
+    ref_o, ref_l = G.oracle_full(q, k, v)
+    G.check_f32(out, lse, ref_o, ref_l, "fp32 tiny")
+
+
+@pytest.mark.parametrize("L,d,mask,window", [
+    (1, 64, "none", 0), (33, 17, "causal", 0), (100, 128, "window", 7),
+    (257, 256, "causal", 0), (300, 1, "window", 0), (129, 96, "none", 0)])
+def test_fp32_ragged(L, d, mask, window):
+    q, k, v = G.rand_qkv(2, 1, L, d, seed=L + d, dtype="f32")
+    out, lse = G.gpu_forward(q, k, v, mask=mask, window=window)
+    ref_o, ref_l = G.oracle_full(q, k, v, mask=mask, window=window)
+    G.check_f32(out, lse, ref_o, ref_l, f"fp32 L={L} d={d} {mask}")
+
+
+# ---------------------------------------------------------------- bf16 path
+SMALL = [
+    (1, 1, 1, 64), (1, 1, 2, 128), (1, 2, 127, 64), (2, 1, 128, 128), (1, 1, 129, 64),
+    (1, 2, 255, 128), (1, 1, 256, 64), (1, 1, 257, 128), (1, 3, 383, 64), (2, 2, 1000, 128),
+    (1, 1, 1025, 64), (1, 1, 2125, 128),
+]
+MASKS = [("none", 0), ("causal", 0), ("window", 0), ("window", 5), ("window", 128),
+         ("window", 300)]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "B{}H{}L{}d{}".format(*s))
+@pytest.mark.parametrize("mask,window", MASKS, ids=lambda m: str(m))
+def test_bf16_small_all_rows(shape, mask, window):
+    B, H, L, d = shape
+    q, k, v = G.rand_qkv(B, H, L, d, seed=L * 7 + d + window)
+    ref_o, ref_l = G.oracle_full(q, k, v, mask=mask, window=window)
+    for bn in (64, 128):
+        out, lse = G.gpu_forward(q, k, v, mask=mask, window=window, block_n=bn)
+        G.check_bf16(out, lse, ref_o, ref_l, f"{shape} {mask}{window} bn={bn}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_bf16_scale_argument(d):
+    q, k, v = G.rand_qkv(1, 2, 300, d, seed=3)
+    for scale in (0.01, 0.3, 1.0):
+        out, lse = G.gpu_forward(q, k, v, mask="causal", scale=scale)
+        ref_o, ref_l = G.oracle_full(q, k, v, mask="causal", scale=scale)
+        G.check_bf16(out, lse, ref_o, ref_l, f"scale {scale}")
+
+
+def test_bf16_many_heads_persistent_schedule():
+    """More work units than SMs, so every CTA walks several units."""
+    q, k, v = G.rand_qkv(3, 37, 600, 64, seed=11)
+    for mask, window in (("causal", 0), ("window", 100), ("none", 0)):
+        out, lse = G.gpu_forward(q, k, v, mask=mask, window=window)
+        ref_o, ref_l = G.oracle_full(q, k, v, mask=mask, window=window)
+        G.check_bf16(out, lse, ref_o, ref_l, f"many heads {mask}")
+
+
+# ---------------------------------------------------------------- full size
+def _sampled(w, block_n=0, per_head=64):
+    q, k, v = ebh.make_qkv(w)
+    BH = w.B * w.H
+    bh_idx, row_idx = ebh.sample_rows(w.L, BH, per_head=per_head)
+    out, lse = G.gpu_forward(q, k, v, mask=w.mask, window=w.window, block_n=block_n)
+    ref_o, ref_l = G.oracle_rows(q, k, v, bh_idx, row_idx, mask=w.mask, window=w.window)
+    o = out.reshape(BH, w.L, w.d)[bh_idx, row_idx]
+    l = lse.reshape(BH, w.L)[bh_idx, row_idx]
+    return (out, lse), G.check_bf16(o, l, ref_o, ref_l, w.name)
+
+
+def test_full_mha_L2048_d64():
+    _sampled(ebh.WORKLOADS["mha_bf16_L2048_d64"])
+
+
+def test_full_mha_L2048_d64_q_times_8_stress():
+    (out, lse), _ = _sampled(ebh.WORKLOADS["mha_bf16_L2048_d64_qx8"])
+    assert np.isfinite(out).all() and np.isfinite(lse).all()
+
+
+def test_full_causal_L8192_block_sizes_agree():
+    w = ebh.WORKLOADS["causal_bf16_L8192_d128"]
+    outs = {}
+    for bn in (64, 128):
+        (out, lse), _ = _sampled(w, block_n=bn, per_head=16 if bn == 64 else 64)
+        outs[bn] = (out, lse)
+    assert np.abs(outs[64][0] - outs[128][0]).max() <= G.BF16_OUT_ATOL
+    assert np.abs(outs[64][1] - outs[128][1]).max() <= G.BF16_LSE_ATOL
+
+
+def test_full_window512_L32768():
+    _sampled(ebh.WORKLOADS["window512_bf16_L32768_d128"])
+
+
+def test_full_causal_L131072_O_of_L_memory():
+    w = ebh.WORKLOADS["causal_bf16_L131072_d128"]
+    q, k, v = ebh.make_qkv(w)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    out = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    ebh.forward(qd, kd, vd, mask="causal", out=out, lse=lse)
+    torch.cuda.synchronize()
+    free_after = torch.cuda.mem_get_info()[0]
+    # no L x L buffer (that would be 550 GB): device memory is unchanged
+    assert abs(free_before - free_after) < (64 << 20)
+    assert ebh.device_status(0) == ebh.ATTN_OK
+    BH = w.B * w.H
+    bh_idx, row_idx = ebh.sample_rows(w.L, BH, per_head=64)
+    ref_o, ref_l = G.oracle_rows(q, k, v, bh_idx, row_idx, mask="causal")
+    o = out.double().cpu().numpy().reshape(BH, w.L, w.d)[bh_idx, row_idx]
+    l = lse.double().cpu().numpy().reshape(BH, w.L)[bh_idx, row_idx]
+    G.check_bf16(o, l, ref_o, ref_l, w.name)
