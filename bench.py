@@ -1,0 +1,478 @@
+"""Benchmark of the exact blockwise attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-sweep] [--cpu-seconds S]
+
+Default workload: the blockwise causal problem B=1, H=32, L=8192, d=128
+(bf16, inputs N(0,1)/sqrt(2)), the configuration the target is stated on.
+One step = one attention forward over the whole problem (one kernel launch).
+Inputs are larger than L2 (3 x 67 MB), so no flush is needed between steps.
+
+Prints one JSON line: value = algorithmic TFLOP/s (4 d x allowed (i, j)
+pairs per head, summed over every rank) over the max-over-ranks device time
+of exactly K steps, plus tokens/s, the roofline of the kernel against the
+measured bf16 peak, the end-to-end number through the public API with host
+buffers, the fp64 CPU oracle timed on a bounded sample (cpu_baseline), SM
+clocks sampled during the timed region, and the pages' own figures as context.
+
+Under torchrun (N > 1) the heads are sharded across ranks (weak scaling: each
+rank runs the full per-GPU problem on its own heads); no collective touches
+the data, only the barrier and the max of the per-rank times.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+METRIC = "attention fwd TFLOP/s and tokens/s (1×B200) vs dense-BF16 roofline, L=2K–128K"
+DEFAULT_WORKLOAD = "causal_bf16_L8192_d128"
+KERNEL_SOURCES = ["exact_blockwise_head_b200/csrc/attn_sm100.cu",
+                  "exact_blockwise_head_b200/csrc/sm100_ptx.cuh",
+                  "exact_blockwise_head_b200/csrc/tiles.h"]
+
+# The pages' own figures: context only, other hardware or none stated.
+CONTEXT = [
+    {"figure": "1250 tokens/s, 15.2 GB", "workload": "L=2048, no blocking",
+     "hardware": "unstated", "page": "Blockwise Parallel Transformer in PyTorch"},
+    {"figure": "836 tokens/s, 18.7 GB", "workload": "L=8192, block 1024",
+     "hardware": "unstated", "page": "Blockwise Parallel Transformer in PyTorch"},
+    {"figure": "721 tokens/s, 12.3 GB", "workload": "L=8192, block 512",
+     "hardware": "unstated", "page": "Blockwise Parallel Transformer in PyTorch"},
+    {"figure": "FlashAttention 3.2x faster, 5x less memory", "workload": "L=4096",
+     "hardware": "RTX 3090",
+     "page": "Attention optimisation strategies for long-sequence inference, sec. 3.1"},
+    {"figure": "78% of theoretical peak", "workload": "8-head attention",
+     "hardware": "A100",
+     "page": "Transformer multi-head attention, 8-head parallel computation, sec. 5.3"},
+]
+
+
+def allowed_pairs(L: int, mask: str, window: int) -> int:
+    """Number of (i, j) pairs the mask allows in one head (closed forms)."""
+    if mask == "none":
+        return L * L
+    if mask == "causal":
+        return L * (L + 1) // 2
+    w = min(window, L - 1)
+    # row i sees keys [max(0, i-w), min(L-1, i+w)]
+    total = L * (2 * w + 1)
+    total -= w * (w + 1)  # clipped at the left edge (rows 0..w-1) and the right edge
+    return total
+
+
+def algorithmic_flops(w) -> float:
+    return 4.0 * w.d * w.B * w.H * allowed_pairs(w.L, w.mask, w.window)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, only if it was
+    taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    ent = rec.get(workload)
+    if not ent or ent.get("kernel_sha") != kernel_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.reasons = 0
+        self.period = period_s
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self._nvml = None
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        s = sorted(self.samples)
+        med = s[len(s) // 2] if s else None
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(s)}
+
+
+def cpu_baseline(w, q, k, v, budget_s: float):
+    """Time the fp64 oracle, as it stands, on a bounded sample of query rows."""
+    import numpy as np
+
+    import oracle
+
+    qf, kf, vf = (t.float().numpy() for t in (q, k, v))
+    BH = w.B * w.H
+    threads = oracle.default_threads()
+    rng = np.random.default_rng(1234)
+
+    def rows_flops(row_idx):
+        total = 0
+        for i in row_idx:
+            i = int(i)
+            if w.mask == "none":
+                n = w.L
+            elif w.mask == "causal":
+                n = i + 1
+            else:
+                n = min(w.L - 1, i + w.window) - max(0, i - w.window) + 1
+            total += 4 * w.d * n
+        return total
+
+    def run(n):
+        bh = rng.integers(0, BH, size=n)
+        rows = rng.integers(0, w.L, size=n)
+        t0 = time.perf_counter()
+        oracle.attention_rows(qf, kf, vf, bh, rows, mask=w.mask, window=w.window,
+                              nthreads=threads)
+        return time.perf_counter() - t0, rows_flops(rows)
+
+    n = max(threads, 8)
+    dt, fl = run(n)
+    while dt < 0.5 and n < 1 << 20:
+        n *= 4
+        dt, fl = run(n)
+    n_final = max(1, int(n * budget_s / max(dt, 1e-6)))
+    dt, fl = run(n_final)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n_final} random query rows of {w.name} (fp64 C oracle, "
+                      f"{threads} threads, {dt:.1f} s)",
+            "rows_per_s": n_final / dt, "tokens_per_s_extrapolated": n_final / dt}
+
+
+def time_gpu(fn, steps, stream, flush=None):
+    """Per-step CUDA-event times (ms) of fn() on `stream`."""
+    import torch
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        if flush is not None:
+            flush()
+        starts[i].record(stream)
+        fn()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+def sweep_other(ebh, torch, names, steps=5, warmup=3):
+    """Kernel-only TFLOP/s of the other workloads (inputs drawn on the GPU)."""
+    res = {}
+    for name in names:
+        w = ebh.WORKLOADS[name]
+        g = torch.Generator(device="cuda").manual_seed(w.seed)
+        shape = (w.B, w.H, w.L, w.d)
+        q, k, v = (torch.randn(shape, device="cuda", generator=g) * w.std for _ in range(3))
+        q = (q * w.q_mult).to(torch.bfloat16)
+        k = k.to(torch.bfloat16)
+        v = v.to(torch.bfloat16)
+        out = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.L), device="cuda", dtype=torch.float32)
+        stream = torch.cuda.current_stream()
+        flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+        def fn():
+            ebh.forward(q, k, v, mask=w.mask, window=w.window, out=out, lse=lse)
+
+        for _ in range(warmup):
+            fn()
+        small = 3 * q.numel() * 2 < 126e6
+        ms = time_gpu(fn, steps, stream, flush=(lambda: flush_buf.zero_()) if small else None)
+        avg = sum(ms) / len(ms)
+        fl = algorithmic_flops(w)
+        res[name] = {"ms": round(avg, 4), "tflops": round(fl / avg / 1e9, 1),
+                     "tokens_per_s": round(w.B * w.L / avg * 1e3, 1),
+                     "l2": "flushed between steps" if small else "inputs larger than L2"}
+        del q, k, v, out, lse, flush_buf
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--block-n", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    import exact_blockwise_head_b200 as ebh
+
+    w = ebh.WORKLOADS[args.workload]
+    if w.dtype != "bf16":
+        ap.error("the bench times the bf16 tensor-core path")
+
+    if args.impl == "reference":
+        return reference_arm(args, w, world, rank)
+
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    from exact_blockwise_head_b200.sharding import weak_scaling_heads
+
+    start, stop = weak_scaling_heads(w.B * w.H, world, rank)
+    # this rank's heads: same shape as the single-GPU problem, own seed
+    wr = w.with_(seed=w.seed + start) if world > 1 else w
+    q, k, v = ebh.make_qkv(wr)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    out = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.H, w.L), device="cuda", dtype=torch.float32)
+    stream = torch.cuda.current_stream()
+    inputs_bytes = 3 * qd.numel() * 2
+    l2_note = "inputs larger than L2 (126 MB)"
+    flush = None
+    if inputs_bytes < 126e6:
+        flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        flush = lambda: flush_buf.zero_()  # noqa: E731
+        l2_note = "L2 flushed between steps (256 MB write, outside the events)"
+
+    def step():
+        ebh.forward(qd, kd, vd, mask=w.mask, window=w.window, block_n=args.block_n, out=out,
+                    lse=lse)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        ms = time_gpu(step, args.steps, stream, flush)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    assert ebh.device_status(local_rank) == ebh.ATTN_OK, "a kernel wait ran out"
+    total_ms = sum(ms)
+    t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    flops_per_step = algorithmic_flops(w) * world
+    ms_per_step = total_ms / args.steps
+    value = flops_per_step / (ms_per_step * 1e-3) / 1e12
+    tokens_per_s = w.B * w.L * world / (ms_per_step * 1e-3)
+
+    # ---- end to end through the public API with host buffers
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    qe, ke, ve = (torch.empty_like(qd) for _ in range(3))
+
+    def e2e_step():
+        qe.copy_(qh, non_blocking=True)
+        ke.copy_(kh, non_blocking=True)
+        ve.copy_(vh, non_blocking=True)
+        ebh.forward(qe, ke, ve, mask=w.mask, window=w.window, block_n=args.block_n, out=out,
+                    lse=lse)
+        oh.copy_(out, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, 20))
+    e2e_ms = time_gpu(e2e_step, e2e_steps, stream)
+    e2e_t = torch.tensor([sum(e2e_ms) / e2e_steps], device="cuda", dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_value = flops_per_step / (float(e2e_t.item()) * 1e-3) / 1e12
+    h2d = 3 * qd.numel() * 2
+    d2h = out.numel() * 2 + lse.numel() * 4
+
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    per_launch_ms = sum(ms) / len(ms)
+    achieved = algorithmic_flops(w) / (per_launch_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "tokens_per_s": round(tokens_per_s, 1),
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
+                   "mask": w.mask, "window": w.window,
+                   "block_n": args.block_n or 128, "heads_per_gpu": w.B * w.H,
+                   "global_heads": w.B * w.H * world, "parallelism": f"heads sharded x{world}",
+                   "l2": l2_note},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)"
+                     if peak_kind == "measured" else "fallback 1.59 PFLOP/s",
+                     "frac_of_spec_2250": round(achieved / SPEC_BF16_TFLOPS, 4),
+                     "frac_of_sustained": round(
+                         achieved / float(peaks.get("bf16_tflops_sustained", 1400.0)), 4),
+                     "traffic": traffic_for(w.name),
+                     "flops_per_launch": algorithmic_flops(w)},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "ms_per_step": round(float(e2e_t.item()), 4)},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "context_only": CONTEXT,
+    }
+    if rank == 0 and not args.no_sweep and world == 1:
+        others = [n for n in ("mha_bf16_L2048_d64", "mha_bf16_L2048_d64_qx8",
+                              "window512_bf16_L32768_d128", "causal_bf16_L131072_d128",
+                              "causal_bf16_L8192_d128")
+                  if n != w.name]
+        del qe, ke, ve
+        line["other_workloads_kernel_only"] = sweep_other(ebh, torch, others)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, q, k, v, args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def reference_arm(args, w, world, rank):
+    """The fp64 CPU oracle as the reference arm: each step is a bounded sample
+    of the workload's query rows, timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return 0
+    import numpy as np
+
+    import exact_blockwise_head_b200 as ebh
+    import oracle
+
+    q, k, v = ebh.make_qkv(w)
+    qf, kf, vf = (t.float().numpy() for t in (q, k, v))
+    threads = oracle.default_threads()
+    rng = np.random.default_rng(99)
+    rows_per_step = 32 * max(threads, 1)
+
+    def step():
+        bh = rng.integers(0, w.B * w.H, size=rows_per_step)
+        rows = rng.integers(0, w.L, size=rows_per_step)
+        oracle.attention_rows(qf, kf, vf, bh, rows, mask=w.mask, window=w.window,
+                              nthreads=threads)
+        return rows
+
+    for _ in range(args.warmup):
+        step()
+    flops = 0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        rows = step()
+        for i in rows:
+            i = int(i)
+            n = w.L if w.mask == "none" else (i + 1 if w.mask == "causal" else
+                                              min(w.L - 1, i + w.window) - max(0, i - w.window)
+                                              + 1)
+            flops += 4 * w.d * n
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "mask": w.mask,
+                   "window": w.window},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows_per_step} random query rows per step of {w.name}"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main() or 0)

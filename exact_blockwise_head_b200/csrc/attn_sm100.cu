@@ -403,7 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!w.valid) continue;
       const int row = w.q_first + r;
       float m_used = -INFINITY;  // running max, log2 units
-      float l = 0.f;             // running sum against m_used
+      float l = 0.f;             // running sum of the probabilities against m_used
+      float lr = 0.f;            // the same sum over the bf16-rounded probabilities
 
       for (int j = w.lo; j < w.hi; ++j) {
         if (!(ok = warp_wait(bar(C::kBarSFull + t), s_cnt & 1, abort_flag, limit))) break;
@@ -442,6 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (m_tile > m_used + kRescaleThreshold) {
           alpha = ex2_approx(m_used - m_tile);
           l *= alpha;
+          lr *= alpha;
           m_used = m_tile;
           rescale = true;
         }
@@ -459,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const float msub = m_used == -INFINITY ? 0.f : m_used;
-        float ls0 = 0.f, ls1 = 0.f;
+        float ls0 = 0.f, ls1 = 0.f, lr0 = 0.f, lr1 = 0.f;
         // P in chunks of 64 keys = 32 packed columns, written over the first
         // half of S_t (those S values are already in registers).
 #pragma unroll
@@ -472,10 +474,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ls0 += p0;
             ls1 += p1;
             pk[c] = pack_bf16x2(p0, p1);
+            lr0 += __uint_as_float(pk[c] << 16);           // bf16 -> f32 is exact
+            lr1 += __uint_as_float(pk[c] & 0xffff0000u);
           }
           tmem_st32(tS + 32 * cc, pk);
         }
         l += ls0 + ls1;
+        lr += lr0 + lr1;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(C::kBarPFull + t));
@@ -486,7 +491,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = warp_wait(bar(C::kBarOFull + t), o_cnt & 1, abort_flag, limit))) break;
       ++o_cnt;
       tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      // O is divided by the sum of exactly the (bf16) weights that multiplied
+      // V, so the weights sum to one; LSE uses the unrounded sum.
+      const float inv_l = lr > 0.f ? 1.f / lr : 0.f;
       const bool row_ok = row < p.L;
       const size_t row_off = (static_cast<size_t>(w.bh) * p.L + (row_ok ? row : 0)) * D;
       uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row_off);
