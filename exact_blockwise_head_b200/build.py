@@ -18,6 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libebh_attn.so")
+TRACE_LIB = os.path.join(PKG, "libebh_attn_trace.so")
 SOURCES = ["api.cpp", "attn_sm100.cu", "attn_f32.cu"]
 HEADERS = ["kernels.h", "sm100_ptx.cuh", "tiles.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -44,22 +45,33 @@ def is_stale() -> bool:
     return any(os.path.getmtime(f) > t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every source into libebh_attn.so (skipped when up to date)."""
-    if not force and not is_stale():
+def build(force: bool = False, verbose: bool = False, trace: bool = False,
+          defines=(), out: str | None = None) -> str:
+    """Compile every source into libebh_attn.so (skipped when up to date).
+
+    trace=True builds the profiling variant libebh_attn_trace.so, whose
+    tensor-core kernel records pipeline timestamps for CTA 0 (read back with
+    attn_pipeline_trace_read).  `defines` are extra -D flags; `out` overrides
+    the output path.
+    """
+    target = out or (TRACE_LIB if trace else LIB)
+    if not force and not defines and out is None and target == LIB and not is_stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = target + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC,-O3,-fvisibility=hidden", "-cudart", "static",
            "-I", INCLUDE, "-I", CSRC, "-o", tmp]
+    if trace:
+        cmd.append("-DEBH_PIPELINE_TRACE")
+    cmd += [f"-D{d}" for d in defines]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
+                trace="--trace" in sys.argv))

@@ -8,7 +8,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/attn.h"
+#include "attn.h"
 #include "kernels.h"
 #include "tiles.h"
 

@@ -37,7 +37,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/attn.h"
+#include "attn.h"
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 #include "tiles.h"
@@ -51,9 +51,62 @@ constexpr int kUnitRows = kBM * kNQ;
 constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kLaunchRegs = 168;   // 65536 / 384 rounded down to a multiple of 8
+constexpr int kSoftmaxRegs = 208;
+constexpr int kOtherRegs = 80;
+static_assert(kSoftmaxRegs * 256 + kOtherRegs * 128 <= kLaunchRegs * kThreads,
+              "register split exceeds the launch allocation");
+// Share of the exponentials computed on the FMA pipe (polynomial) instead of
+// the MUFU pipe, on tiles without masked elements: one pair in kPolyEvery
+// (0 = none).
+#ifndef EBH_POLY_EVERY
+#define EBH_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = EBH_POLY_EVERY;
 // Lazy rescale: keep the stale max until the row max exceeds it by more than
 // 2^8 (probabilities then stay <= 256, far inside fp32/bf16 range).
 constexpr float kRescaleThreshold = 8.0f;
+// Compute a tile's exponentials against the stale max before its row max is
+// known (redo the tile when the max outgrew the threshold).  Needs the whole
+// score row live during the exponentials.
+#ifndef EBH_SPECULATE
+#define EBH_SPECULATE 0
+#endif
+constexpr bool kSpeculate = EBH_SPECULATE;
+// Row-max reduction: independent chains of three-input maxima (0 = a tree).
+#ifndef EBH_MAX_CHAINS
+#define EBH_MAX_CHAINS 4
+#endif
+constexpr int kMaxChains = EBH_MAX_CHAINS;
+
+// Pipeline trace for profiling builds (-DEBH_PIPELINE_TRACE): lane 0 of each
+// warp of CTA 0 appends (event << 56 | key block << 40 | clock64) records to
+// g_pipeline_trace[warp]; attn_pipeline_trace_read() copies them out.
+enum : int {
+  kEvSWait = 1, kEvSReady = 2, kEvSLoaded = 3, kEvMaxDone = 4, kEvPWritten = 5, kEvMasked = 8,
+  kEvEpilogue = 6, kEvEpilogueDone = 7,
+  kEvKWait = 10, kEvKReady = 11, kEvVWait = 16, kEvVReady = 17,
+  kEvPWait = 13, kEvPReady = 14  // + 10 * Q tile
+};
+#ifdef EBH_PIPELINE_TRACE
+constexpr int kTraceLen = 8192;
+__device__ unsigned long long g_pipeline_trace[16][kTraceLen];
+#define EBH_TRACE_COUNTER int tr_n = 0
+#define EBH_TRACE(ev, jj)                                                               \
+  do {                                                                                  \
+    if (blockIdx.x == 0 && (threadIdx.x % 32) == 0 && tr_n < kTraceLen)                 \
+      g_pipeline_trace[threadIdx.x / 32][tr_n++] =                                      \
+          ((unsigned long long)(ev) << 56) | ((unsigned long long)((jj)&0xFFFF) << 40) | \
+          (clock64() & 0xFFFFFFFFFFull);                                                \
+  } while (0)
+#else
+#define EBH_TRACE_COUNTER \
+  do {                    \
+  } while (0)
+#define EBH_TRACE(ev, jj) \
+  do {                    \
+  } while (0)
+#endif
 
 template <int D, int BN>
 struct Cfg {
@@ -182,6 +235,112 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
+// O_t row *= alpha for this warp's 32 rows (tensor memory round trip).  The
+// caller guarantees no MMA is writing O_t (its previous P.V product was issued
+// before the S_t product the caller has waited for, and they complete in order).
+template <int D>
+__device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    tmem_ld32(tO + 32 * c, o);
+    tmem_wait_ld();
+    reg_fence32(o);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+    tmem_st32(tO + 32 * c, o);
+  }
+}
+
+// Max of n values by a tree of three-input maxima (depth log3 n).
+template <int N>
+struct TreeMax {
+  static __device__ __forceinline__ float run(float* v) {
+    constexpr int M = (N + 2) / 3;
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+      if (3 * i + 2 < N) v[i] = max3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+      else if (3 * i + 1 < N) v[i] = fmaxf(v[3 * i], v[3 * i + 1]);
+      else v[i] = v[3 * i];
+    }
+    return TreeMax<M>::run(v);
+  }
+};
+template <>
+struct TreeMax<1> {
+  static __device__ __forceinline__ float run(float* v) { return v[0]; }
+};
+
+// Max of one row of a score tile: kMaxChains independent chains of
+// three-input maxima, or (kMaxChains == 0) a tree.
+template <int BN>
+__device__ __forceinline__ float row_max(const float* s) {
+  if constexpr (kMaxChains == 0) {
+    constexpr int M = (BN + 2) / 3;
+    float v[M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+      if (3 * i + 2 < BN) v[i] = max3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
+      else if (3 * i + 1 < BN) v[i] = fmaxf(s[3 * i], s[3 * i + 1]);
+      else v[i] = s[3 * i];
+    }
+    return TreeMax<M>::run(v);
+  } else {
+    constexpr int K = kMaxChains;
+    float m[K];
+#pragma unroll
+    for (int i = 0; i < K; ++i) m[i] = fmaxf(s[i], s[i + K]);
+#pragma unroll
+    for (int c = 2 * K; c < BN; c += 2 * K) {
+#pragma unroll
+      for (int i = 0; i < K; ++i) m[i] = max3(m[i], s[c + i], s[c + K + i]);
+    }
+    return TreeMax<K>::run(m);
+  }
+}
+
+// p_c = 2^(s_c * cl2 - msub) for one row of a score tile, written to tensor
+// memory as packed bf16 over the first half of the tile's S columns (those
+// scores are already in registers), 32 keys at a time.  l accumulates the
+// probabilities, lr the bf16-rounded probabilities the P.V product will use.
+// kPoly: compute one pair in kPolyEvery on the FMA pipe (tiles without masked
+// elements only: the polynomial has no -inf handling).
+template <int BN, bool kPoly>
+__device__ __forceinline__ void write_probabilities(const float* s, float cl2, float msub,
+                                                    uint32_t tS, float& l, float& lr) {
+  float la = 0.f, lb = 0.f, lc = 0.f, ld = 0.f;
+  float ra = 0.f, rb = 0.f, rc = 0.f, rd = 0.f;
+#pragma unroll
+  for (int cc = 0; cc < BN / 32; ++cc) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int e = 32 * cc + 2 * c;
+      float x0, x1, p0, p1;
+      fma2(x0, x1, s[e], s[e + 1], cl2, cl2, -msub, -msub);
+      bool poly = false;
+      if constexpr (kPoly) poly = (c % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+      if (poly) {
+        exp2_poly2(x0, x1, p0, p1);
+      } else {
+        p0 = ex2_approx(x0);
+        p1 = ex2_approx(x1);
+      }
+      pk[c] = pack_bf16x2(p0, p1);
+      if (c & 1) {
+        add2(lc, ld, lc, ld, p0, p1);
+        acc_bf16x2(rc, rd, pk[c]);
+      } else {
+        add2(la, lb, la, lb, p0, p1);
+        acc_bf16x2(ra, rb, pk[c]);
+      }
+    }
+    tmem_st16(tS + 16 * cc, pk);
+  }
+  l += (la + lb) + (lc + ld);
+  lr += (ra + rb) + (rc + rd);
+}
+
 template <int D, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -233,161 +392,178 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
   const uint64_t limit = p.timeout_ns;
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int kv_it = 0;
-      int q_cnt[kNQ] = {0, 0};
-      bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-        const Unit w = decode_unit<BN>(u, p);
-        auto load_q = [&](int t) -> bool {
-          if (!w.valid[t]) return true;
-          if (!wait_bounded(bar(C::kBarQEmpty + t), (q_cnt[t] & 1) ^ 1, abort_flag, limit))
+  // Registers: the softmax warpgroups hold a 128-wide score row per thread;
+  // the producer / MMA warpgroup needs few.  kSoftmaxRegs * 256 +
+  // kOtherRegs * 128 must not exceed the launch's kLaunchRegs * 384 (checked
+  // on the host before launch), or the grow would wait forever.  Each role
+  // runs inside the branch that set its register count, so the compiler
+  // allocates each role's code under its own limit.
+  if (warp >= 8) {
+    regs_shrink<kOtherRegs>();
+    if (warp == kProducerWarp) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0) {
+        int kv_it = 0;
+        int q_cnt[kNQ] = {0, 0};
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+          const Unit w = decode_unit<BN>(u, p);
+          auto load_q = [&](int t) -> bool {
+            if (!w.valid[t]) return true;
+            if (!wait_bounded(bar(C::kBarQEmpty + t), (q_cnt[t] & 1) ^ 1, abort_flag, limit))
+              return false;
+            mbar_arrive_expect_tx(bar(C::kBarQFull + t), C::kQTileBytes);
+            const uint32_t dst = smem_addr(sQ + t * C::kQTileBytes);
+  #pragma unroll
+            for (int c = 0; c < C::kDChunks; ++c)
+              tma_load_3d(dst + c * kBM * 128, &tm_q, bar(C::kBarQFull + t), c * 64, w.q_first[t],
+                          w.bh);
+            ++q_cnt[t];
+            return true;
+          };
+          ok = load_q(0) && load_q(1);
+          for (int j = w.ulo; ok && j < w.uhi; ++j) {
+  #pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+              const int s = kv_it % C::kStages;
+              ok = wait_bounded(bar(C::kBarKVEmpty + s), ((kv_it / C::kStages) & 1) ^ 1, abort_flag,
+                                limit);
+              if (!ok) break;
+              mbar_arrive_expect_tx(bar(C::kBarKVFull + s), C::kKVTileBytes);
+              const uint32_t dst = smem_addr(sKV + s * C::kKVTileBytes);
+              const CUtensorMap* map = which == 0 ? &tm_k : &tm_v;
+  #pragma unroll
+              for (int c = 0; c < C::kDChunks; ++c)
+                tma_load_3d(dst + c * BN * 128, map, bar(C::kBarKVFull + s), c * 64, j * BN, w.bh);
+              ++kv_it;
+            }
+          }
+        }
+        // Every load this thread issued must land before the CTA may exit.
+        for (int s = 0; s < C::kStages; ++s) {
+          if (kv_it > s) {
+            const int last = s + C::kStages * ((kv_it - 1 - s) / C::kStages);
+            drain_wait(bar(C::kBarKVFull + s), (last / C::kStages) & 1, limit);
+          }
+        }
+        for (int t = 0; t < kNQ; ++t)
+          if (q_cnt[t] > 0) drain_wait(bar(C::kBarQFull + t), (q_cnt[t] - 1) & 1, limit);
+      }
+    } else if (warp == kMmaWarp) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, BN, false);
+        constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, true);
+        int kv_it = 0;
+        int q_cnt[kNQ] = {0, 0}, p_cnt[kNQ] = {0, 0}, o_cnt[kNQ] = {0, 0};
+        bool ok = true;
+        EBH_TRACE_COUNTER;
+
+        auto issue_s = [&](int t, int kst) {
+          const uint32_t qa = smem_addr(sQ + t * C::kQTileBytes);
+          const uint32_t kb = smem_addr(sKV + kst * C::kKVTileBytes);
+  #pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint64_t a = sdesc_sw128(qa + (k / 4) * kBM * 128 + (k % 4) * 32, 16, 1024);
+            const uint64_t b = sdesc_sw128(kb + (k / 4) * BN * 128 + (k % 4) * 32, 16, 1024);
+            mma_ss(tmem + C::kColS + t * BN, a, b, idesc_s, k > 0 ? 1u : 0u);
+          }
+        };
+        auto issue_pv = [&](int t, int vst, bool first) -> bool {
+          EBH_TRACE(kEvPWait + 10 * t, 0);
+          if (!wait_bounded(bar(C::kBarPFull + t), p_cnt[t] & 1, abort_flag, limit)) return false;
+          EBH_TRACE(kEvPReady + 10 * t, 0);
+          ++p_cnt[t];
+          if (first &&
+              !wait_bounded(bar(C::kBarOEmpty + t), (o_cnt[t] & 1) ^ 1, abort_flag, limit))
             return false;
-          mbar_arrive_expect_tx(bar(C::kBarQFull + t), C::kQTileBytes);
-          const uint32_t dst = smem_addr(sQ + t * C::kQTileBytes);
-#pragma unroll
-          for (int c = 0; c < C::kDChunks; ++c)
-            tma_load_3d(dst + c * kBM * 128, &tm_q, bar(C::kBarQFull + t), c * 64, w.q_first[t],
-                        w.bh);
-          ++q_cnt[t];
+          tc_fence_after();
+          const uint32_t vb = smem_addr(sKV + vst * C::kKVTileBytes);
+  #pragma unroll
+          for (int k = 0; k < BN / 16; ++k) {
+            const uint64_t b = sdesc_sw128(vb + k * 16 * 128, BN * 128, 1024);
+            mma_ts(tmem + C::kColO + t * D, tmem + C::kColS + t * BN + k * 8, b, idesc_o,
+                   (first && k == 0) ? 0u : 1u);
+          }
           return true;
         };
-        ok = load_q(0) && load_q(1);
-        for (int j = w.ulo; ok && j < w.uhi; ++j) {
-#pragma unroll 1
-          for (int which = 0; which < 2; ++which) {
-            const int s = kv_it % C::kStages;
-            ok = wait_bounded(bar(C::kBarKVEmpty + s), ((kv_it / C::kStages) & 1) ^ 1, abort_flag,
-                              limit);
-            if (!ok) break;
-            mbar_arrive_expect_tx(bar(C::kBarKVFull + s), C::kKVTileBytes);
-            const uint32_t dst = smem_addr(sKV + s * C::kKVTileBytes);
-            const CUtensorMap* map = which == 0 ? &tm_k : &tm_v;
-#pragma unroll
-            for (int c = 0; c < C::kDChunks; ++c)
-              tma_load_3d(dst + c * BN * 128, map, bar(C::kBarKVFull + s), c * 64, j * BN, w.bh);
+
+        for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+          const Unit w = decode_unit<BN>(u, p);
+          int pend_v = -1;  // ring stage of V_(j-1) still owed a P_1 . V product
+          for (int j = w.ulo; ok && j < w.uhi; ++j) {
+            const int kst = kv_it % C::kStages;
+            const uint32_t kph = (kv_it / C::kStages) & 1;
             ++kv_it;
+            const int vst = kv_it % C::kStages;
+            const uint32_t vph = (kv_it / C::kStages) & 1;
+            ++kv_it;
+            EBH_TRACE(kEvKWait, j);
+            if (!(ok = wait_bounded(bar(C::kBarKVFull + kst), kph, abort_flag, limit))) break;
+            EBH_TRACE(kEvKReady, j);
+            const bool in0 = in_range(w, 0, j), in1 = in_range(w, 1, j);
+            if (in0) {
+              if (j == w.lo[0] &&
+                  !(ok = wait_bounded(bar(C::kBarQFull + 0), q_cnt[0] & 1, abort_flag, limit)))
+                break;
+              tc_fence_after();
+              issue_s(0, kst);
+              mma_commit(bar(C::kBarSFull + 0));
+              if (j == w.hi[0] - 1) mma_commit(bar(C::kBarQEmpty + 0));
+            }
+            if (pend_v >= 0) {
+              if (!(ok = issue_pv(1, pend_v, j - 1 == w.lo[1]))) break;
+              mma_commit(bar(C::kBarKVEmpty + pend_v));
+              if (j - 1 == w.hi[1] - 1) mma_commit(bar(C::kBarOFull + 1));
+              pend_v = -1;
+            }
+            if (in1) {
+              if (j == w.lo[1] &&
+                  !(ok = wait_bounded(bar(C::kBarQFull + 1), q_cnt[1] & 1, abort_flag, limit)))
+                break;
+              tc_fence_after();
+              issue_s(1, kst);
+              mma_commit(bar(C::kBarSFull + 1));
+              if (j == w.hi[1] - 1) mma_commit(bar(C::kBarQEmpty + 1));
+            }
+            mma_commit(bar(C::kBarKVEmpty + kst));  // K_j no longer needed
+            EBH_TRACE(kEvVWait, j);
+            if (!(ok = wait_bounded(bar(C::kBarKVFull + vst), vph, abort_flag, limit))) break;
+            EBH_TRACE(kEvVReady, j);
+            if (in0) {
+              if (!(ok = issue_pv(0, vst, j == w.lo[0]))) break;
+              if (j == w.hi[0] - 1) mma_commit(bar(C::kBarOFull + 0));
+            }
+            if (in1) {
+              pend_v = vst;
+            } else {
+              mma_commit(bar(C::kBarKVEmpty + vst));
+            }
+          }
+          if (ok && pend_v >= 0) {
+            const int j = w.uhi;
+            if ((ok = issue_pv(1, pend_v, j - 1 == w.lo[1]))) {
+              mma_commit(bar(C::kBarKVEmpty + pend_v));
+              if (j - 1 == w.hi[1] - 1) mma_commit(bar(C::kBarOFull + 1));
+            }
+          }
+          if (w.valid[0]) {
+            ++q_cnt[0];
+            ++o_cnt[0];
+          }
+          if (w.valid[1]) {
+            ++q_cnt[1];
+            ++o_cnt[1];
           }
         }
+        // No MMA may still be writing tensor memory when it is freed.
+        mma_commit(bar(C::kBarDrain));
+        drain_wait(bar(C::kBarDrain), 0, limit);
       }
-      // Every load this thread issued must land before the CTA may exit.
-      for (int s = 0; s < C::kStages; ++s) {
-        if (kv_it > s) {
-          const int last = s + C::kStages * ((kv_it - 1 - s) / C::kStages);
-          drain_wait(bar(C::kBarKVFull + s), (last / C::kStages) & 1, limit);
-        }
-      }
-      for (int t = 0; t < kNQ; ++t)
-        if (q_cnt[t] > 0) drain_wait(bar(C::kBarQFull + t), (q_cnt[t] - 1) & 1, limit);
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, BN, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, true);
-      int kv_it = 0;
-      int q_cnt[kNQ] = {0, 0}, p_cnt[kNQ] = {0, 0}, o_cnt[kNQ] = {0, 0};
-      bool ok = true;
-
-      auto issue_s = [&](int t, int kst) {
-        const uint32_t qa = smem_addr(sQ + t * C::kQTileBytes);
-        const uint32_t kb = smem_addr(sKV + kst * C::kKVTileBytes);
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint64_t a = sdesc_sw128(qa + (k / 4) * kBM * 128 + (k % 4) * 32, 16, 1024);
-          const uint64_t b = sdesc_sw128(kb + (k / 4) * BN * 128 + (k % 4) * 32, 16, 1024);
-          mma_ss(tmem + C::kColS + t * BN, a, b, idesc_s, k > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int t, int vst, bool first) -> bool {
-        if (!wait_bounded(bar(C::kBarPFull + t), p_cnt[t] & 1, abort_flag, limit)) return false;
-        ++p_cnt[t];
-        if (first &&
-            !wait_bounded(bar(C::kBarOEmpty + t), (o_cnt[t] & 1) ^ 1, abort_flag, limit))
-          return false;
-        tc_fence_after();
-        const uint32_t vb = smem_addr(sKV + vst * C::kKVTileBytes);
-#pragma unroll
-        for (int k = 0; k < BN / 16; ++k) {
-          const uint64_t b = sdesc_sw128(vb + k * 16 * 128, BN * 128, 1024);
-          mma_ts(tmem + C::kColO + t * D, tmem + C::kColS + t * BN + k * 8, b, idesc_o,
-                 (first && k == 0) ? 0u : 1u);
-        }
-        return true;
-      };
-
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-        const Unit w = decode_unit<BN>(u, p);
-        int pend_v = -1;  // ring stage of V_(j-1) still owed a P_1 . V product
-        for (int j = w.ulo; ok && j < w.uhi; ++j) {
-          const int kst = kv_it % C::kStages;
-          const uint32_t kph = (kv_it / C::kStages) & 1;
-          ++kv_it;
-          const int vst = kv_it % C::kStages;
-          const uint32_t vph = (kv_it / C::kStages) & 1;
-          ++kv_it;
-          if (!(ok = wait_bounded(bar(C::kBarKVFull + kst), kph, abort_flag, limit))) break;
-          const bool in0 = in_range(w, 0, j), in1 = in_range(w, 1, j);
-          if (in0) {
-            if (j == w.lo[0] &&
-                !(ok = wait_bounded(bar(C::kBarQFull + 0), q_cnt[0] & 1, abort_flag, limit)))
-              break;
-            tc_fence_after();
-            issue_s(0, kst);
-            mma_commit(bar(C::kBarSFull + 0));
-            if (j == w.hi[0] - 1) mma_commit(bar(C::kBarQEmpty + 0));
-          }
-          if (pend_v >= 0) {
-            if (!(ok = issue_pv(1, pend_v, j - 1 == w.lo[1]))) break;
-            mma_commit(bar(C::kBarKVEmpty + pend_v));
-            if (j - 1 == w.hi[1] - 1) mma_commit(bar(C::kBarOFull + 1));
-            pend_v = -1;
-          }
-          if (in1) {
-            if (j == w.lo[1] &&
-                !(ok = wait_bounded(bar(C::kBarQFull + 1), q_cnt[1] & 1, abort_flag, limit)))
-              break;
-            tc_fence_after();
-            issue_s(1, kst);
-            mma_commit(bar(C::kBarSFull + 1));
-            if (j == w.hi[1] - 1) mma_commit(bar(C::kBarQEmpty + 1));
-          }
-          mma_commit(bar(C::kBarKVEmpty + kst));  // K_j no longer needed
-          if (!(ok = wait_bounded(bar(C::kBarKVFull + vst), vph, abort_flag, limit))) break;
-          if (in0) {
-            if (!(ok = issue_pv(0, vst, j == w.lo[0]))) break;
-            if (j == w.hi[0] - 1) mma_commit(bar(C::kBarOFull + 0));
-          }
-          if (in1) {
-            pend_v = vst;
-          } else {
-            mma_commit(bar(C::kBarKVEmpty + vst));
-          }
-        }
-        if (ok && pend_v >= 0) {
-          const int j = w.uhi;
-          if ((ok = issue_pv(1, pend_v, j - 1 == w.lo[1]))) {
-            mma_commit(bar(C::kBarKVEmpty + pend_v));
-            if (j - 1 == w.hi[1] - 1) mma_commit(bar(C::kBarOFull + 1));
-          }
-        }
-        if (w.valid[0]) {
-          ++q_cnt[0];
-          ++o_cnt[0];
-        }
-        if (w.valid[1]) {
-          ++q_cnt[1];
-          ++o_cnt[1];
-        }
-      }
-      // No MMA may still be writing tensor memory when it is freed.
-      mma_commit(bar(C::kBarDrain));
-      drain_wait(bar(C::kBarDrain), 0, limit);
-    }
-  } else if (warp < 8) {
+  } else {
     // ------------------------------------------------------------ softmax
+    regs_grow<kSoftmaxRegs>();
     const int t = warp / 4;
     const int wq = warp % 4;                 // this warp's 32-lane slice of tensor memory
     const int r = threadIdx.x % kBM;         // query row within the Q tile
@@ -397,6 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float cl2 = p.scale_log2;
     int s_cnt = 0, o_cnt = 0;
     bool ok = true;
+    EBH_TRACE_COUNTER;
 
     for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
       const TileWork w = decode_tile<BN>(u, t, p);
@@ -407,7 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float lr = 0.f;            // the same sum over the bf16-rounded probabilities
 
       for (int j = w.lo; j < w.hi; ++j) {
+        EBH_TRACE(kEvSWait, j);
         if (!(ok = warp_wait(bar(C::kBarSFull + t), s_cnt & 1, abort_flag, limit))) break;
+        EBH_TRACE(kEvSReady, j);
         ++s_cnt;
         tc_fence_after();
         uint32_t sr[BN];
@@ -417,77 +596,74 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) reg_fence32(sr + 32 * c);
         float* s = reinterpret_cast<float*>(sr);
+        EBH_TRACE(kEvSLoaded, j);
 
-        if (kv_tile_class(p.L, w.q_first, w.q_last, j, p.mask_kind, p.window, BN) !=
-            kTileFull) {
+        const bool full =
+            kv_tile_class(p.L, w.q_first, w.q_last, j, p.mask_kind, p.window, BN) == kTileFull;
+        if (!full) {
           int c_lo, c_hi;
           row_allowed_cols(p.L, row, j, p.mask_kind, p.window, BN, c_lo, c_hi);
 #pragma unroll
           for (int c = 0; c < BN; ++c)
             if (c < c_lo || c >= c_hi) s[c] = -INFINITY;
         }
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-        for (int c = 4; c < BN; c += 4) {
-          mx0 = fmaxf(mx0, s[c]);
-          mx1 = fmaxf(mx1, s[c + 1]);
-          mx2 = fmaxf(mx2, s[c + 2]);
-          mx3 = fmaxf(mx3, s[c + 3]);
-        }
-        const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * cl2;
-        float alpha = 1.f;
-        bool rescale = false;
-        if (m_used == -INFINITY) {
-          // nothing accumulated for this row yet (l == 0 and its O row is 0)
-          m_used = m_tile;
-        } else if (m_tile > m_used + kRescaleThreshold) {
-          alpha = ex2_approx(m_used - m_tile);
-          l *= alpha;
-          lr *= alpha;
-          m_used = m_tile;
-          rescale = true;
-        }
-        if (__any_sync(0xffffffffu, rescale)) {
-          // O_t's previous product is complete (it was issued before S_t(j)).
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * c, o);
-            tmem_wait_ld();
-            reg_fence32(o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tO + 32 * c, o);
+        EBH_TRACE(kEvMasked, j);
+        const float m_tile = row_max<BN>(s) * cl2;
+        if (!kSpeculate || m_used == -INFINITY) {
+          float alpha = 1.f;
+          bool rescale = false;
+          if (m_used == -INFINITY) {
+            // nothing accumulated for this row yet (l == 0 and its O row is 0)
+            m_used = m_tile;
+          } else if (m_tile > m_used + kRescaleThreshold) {
+            alpha = ex2_approx(m_used - m_tile);
+            l *= alpha;
+            lr *= alpha;
+            m_used = m_tile;
+            rescale = true;
+          }
+          if (__any_sync(0xffffffffu, rescale)) rescale_o_row<D>(tO, alpha);
+          const float msub = m_used == -INFINITY ? 0.f : m_used;
+          EBH_TRACE(kEvMaxDone, j);
+          if (full) {
+            write_probabilities<BN, (kPolyEvery > 0)>(s, cl2, msub, tS, l, lr);
+          } else {
+            write_probabilities<BN, false>(s, cl2, msub, tS, l, lr);
+          }
+        } else {
+          // Speculate that the stale reference m_used still holds (the tile
+          // max exceeds it by at most the threshold), so the exponentials do
+          // not wait for the max; if it does not hold for some row, redo the
+          // tile against the new max and rescale that row of O.
+          const float l0 = l, lr0 = lr;
+          EBH_TRACE(kEvMaxDone, j);
+          if (full) {
+            write_probabilities<BN, (kPolyEvery > 0)>(s, cl2, m_used, tS, l, lr);
+          } else {
+            write_probabilities<BN, false>(s, cl2, m_used, tS, l, lr);
+          }
+          const bool redo = m_tile > m_used + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, redo)) {
+            float alpha = 1.f;
+            if (redo) {
+              alpha = ex2_approx(m_used - m_tile);
+              m_used = m_tile;
+            }
+            l = l0 * alpha;
+            lr = lr0 * alpha;
+            rescale_o_row<D>(tO, alpha);
+            write_probabilities<BN, false>(s, cl2, m_used, tS, l, lr);
           }
         }
-        const float msub = m_used == -INFINITY ? 0.f : m_used;
-        float ls0 = 0.f, ls1 = 0.f, lr0 = 0.f, lr1 = 0.f;
-        // P in chunks of 64 keys = 32 packed columns, written over the first
-        // half of S_t (those S values are already in registers).
-#pragma unroll
-        for (int cc = 0; cc < BN / 64; ++cc) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2_approx(fmaf(s[64 * cc + 2 * c], cl2, -msub));
-            const float p1 = ex2_approx(fmaf(s[64 * cc + 2 * c + 1], cl2, -msub));
-            ls0 += p0;
-            ls1 += p1;
-            pk[c] = pack_bf16x2(p0, p1);
-            lr0 += __uint_as_float(pk[c] << 16);           // bf16 -> f32 is exact
-            lr1 += __uint_as_float(pk[c] & 0xffff0000u);
-          }
-          tmem_st32(tS + 32 * cc, pk);
-        }
-        l += ls0 + ls1;
-        lr += lr0 + lr1;
         tmem_wait_st();
         tc_fence_before();
+        EBH_TRACE(kEvPWritten, j);
         mbar_arrive(bar(C::kBarPFull + t));
       }
       if (!ok) break;
 
       // ---- epilogue: O / l -> bf16, LSE = ln 2 * (m + log2 l)
+      EBH_TRACE(kEvEpilogue, 0);
       if (!(ok = warp_wait(bar(C::kBarOFull + t), o_cnt & 1, abort_flag, limit))) break;
       ++o_cnt;
       tc_fence_after();
@@ -519,6 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.lse[static_cast<size_t>(w.bh) * p.L + row] = lse;
       }
       tc_fence_before();
+      EBH_TRACE(kEvEpilogueDone, 0);
       mbar_arrive(bar(C::kBarOEmpty + t));
     }
   }
@@ -621,6 +798,14 @@ int launch_t(const FwdArgs& a, cudaStream_t stream, cudaError_t* err) {
       *err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   C::kSmemBytes);
       if (*err != cudaSuccess) return ATTN_ERR_CUDA;
+      // The in-kernel register split assumes exactly kLaunchRegs per thread
+      // at launch; refuse to launch a build where that does not hold.
+      cudaFuncAttributes fa;
+      if ((*err = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess) return ATTN_ERR_CUDA;
+      if (fa.numRegs != kLaunchRegs) {
+        *err = cudaErrorInvalidConfiguration;
+        return ATTN_ERR_CUDA;
+      }
       attr_set[device] = true;
     }
   }
@@ -689,3 +874,16 @@ int read_device_status(int device, int reset, cudaError_t* err) {
 }
 
 }  // namespace ebh
+
+#ifdef EBH_PIPELINE_TRACE
+// Profiling builds only: copy out / clear the pipeline trace of CTA 0.
+extern "C" __attribute__((visibility("default"))) int attn_pipeline_trace_read(
+    unsigned long long* host) {
+  return static_cast<int>(
+      cudaMemcpyFromSymbol(host, ebh::g_pipeline_trace, sizeof(ebh::g_pipeline_trace)));
+}
+extern "C" __attribute__((visibility("default"))) int attn_pipeline_trace_clear() {
+  static unsigned long long zero[16][ebh::kTraceLen];
+  return static_cast<int>(cudaMemcpyToSymbol(ebh::g_pipeline_trace, zero, sizeof(zero)));
+}
+#endif

@@ -225,7 +225,96 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------- registers
+// Move registers between warpgroups (all warps of a warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void regs_grow() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_shrink() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- math
+// Paired fp32 arithmetic: one instruction updates two lanes' worth of values
+// (d0, d1) = (a0, a1) op (b0, b1).
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.ftz.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.ftz.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// Same, rounding toward -inf.
+__device__ __forceinline__ void add2_rm(float& d0, float& d1, float a0, float a1, float b0,
+                                        float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rm.ftz.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void sub2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.ftz.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// max of three
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// (a, b) += the two bf16 halves of `pk` (low half to a), each widened exactly.
+__device__ __forceinline__ void acc_bf16x2(float& a, float& b, uint32_t pk) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "r"(pk));
+}
+
+// 2^x on the FMA pipe for two values (relieves the MUFU pipe, which would
+// otherwise bound the softmax).  Cody-Waite style range reduction,
+// x = j + f with j = floor(x) and f in [0, 1), then 2^f from a degree-3
+// polynomial and 2^j by adding j to the exponent field.  The coefficients are
+// this project's own Remez fit of 2^f on [0, 1) in relative error (see
+// fit_exp2_poly.py beside this file): max relative error 7.5e-5, far below the
+// 2^-9 of the bf16 rounding applied to the probabilities.  Inputs are clamped
+// at -126, so the result is a normal float; values below 2^-126 come out as
+// ~2^-126 instead of smaller, which no sum can notice.  Requires x <= 127.
+constexpr float kExp2C0 = 0x1.fff632p-1f;  // 0.99992520
+constexpr float kExp2C1 = 0x1.64444cp-1f;  // 0.69583356
+constexpr float kExp2C2 = 0x1.cefc4cp-3f;  // 0.22606716
+constexpr float kExp2C3 = 0x1.3f96a4p-4f;  // 0.07802452
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: adding it leaves the integer in the mantissa
+
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0, t1, j0, j1, f0, f1, q0, q1;
+  add2_rm(t0, t1, x0, x1, kRoundMagic, kRoundMagic);  // magic + floor(x), exact
+  sub2(j0, j1, t0, t1, kRoundMagic, kRoundMagic);     // floor(x)
+  sub2(f0, f1, x0, x1, j0, j1);                       // f in [0, 1)
+  fma2(q0, q1, kExp2C3, kExp2C3, f0, f1, kExp2C2, kExp2C2);
+  fma2(q0, q1, q0, q1, f0, f1, kExp2C1, kExp2C1);
+  fma2(q0, q1, q0, q1, f0, f1, kExp2C0, kExp2C0);
+  // the low mantissa bits of t hold floor(x); shifted by 23 they land in the
+  // exponent field (the magic's own bits shift out of the word)
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
