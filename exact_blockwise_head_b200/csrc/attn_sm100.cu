@@ -48,36 +48,19 @@ namespace {
 constexpr int kBM = 128;          // query rows per Q tile (= tensor-memory lanes)
 constexpr int kNQ = 2;            // Q tiles per work unit
 constexpr int kUnitRows = kBM * kNQ;
-constexpr int kThreads = 384;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kLaunchRegs = 168;   // 65536 / 384 rounded down to a multiple of 8
-constexpr int kSoftmaxRegs = 208;
-constexpr int kOtherRegs = 80;
-static_assert(kSoftmaxRegs * 256 + kOtherRegs * 128 <= kLaunchRegs * kThreads,
+constexpr int kSoftmaxWarps = 8;   // per Q tile: two per tensor-memory sub-partition
+constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
+constexpr int kThreads = (kNQ * kSoftmaxWarps + 4) * 32;  // + producer, MMA, 2 idle
+constexpr int kProducerWarp = kNQ * kSoftmaxWarps;
+constexpr int kMmaWarp = kProducerWarp + 1;
+constexpr int kLaunchRegs = 96;    // 65536 / 640 rounded down to a multiple of 8
+constexpr int kSoftmaxRegs = 104;
+constexpr int kOtherRegs = 64;
+static_assert(kSoftmaxRegs * kNQ * kSoftmaxThreads + kOtherRegs * 128 <= kLaunchRegs * kThreads,
               "register split exceeds the launch allocation");
-// Share of the exponentials computed on the FMA pipe (polynomial) instead of
-// the MUFU pipe, on tiles without masked elements: one pair in kPolyEvery
-// (0 = none).
-#ifndef EBH_POLY_EVERY
-#define EBH_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = EBH_POLY_EVERY;
 // Lazy rescale: keep the stale max until the row max exceeds it by more than
 // 2^8 (probabilities then stay <= 256, far inside fp32/bf16 range).
 constexpr float kRescaleThreshold = 8.0f;
-// Compute a tile's exponentials against the stale max before its row max is
-// known (redo the tile when the max outgrew the threshold).  Needs the whole
-// score row live during the exponentials.
-#ifndef EBH_SPECULATE
-#define EBH_SPECULATE 0
-#endif
-constexpr bool kSpeculate = EBH_SPECULATE;
-// Row-max reduction: independent chains of three-input maxima (0 = a tree).
-#ifndef EBH_MAX_CHAINS
-#define EBH_MAX_CHAINS 4
-#endif
-constexpr int kMaxChains = EBH_MAX_CHAINS;
 
 // Pipeline trace for profiling builds (-DEBH_PIPELINE_TRACE): lane 0 of each
 // warp of CTA 0 appends (event << 56 | key block << 40 | clock64) records to
@@ -86,11 +69,12 @@ enum : int {
   kEvSWait = 1, kEvSReady = 2, kEvSLoaded = 3, kEvMaxDone = 4, kEvPWritten = 5, kEvMasked = 8,
   kEvEpilogue = 6, kEvEpilogueDone = 7,
   kEvKWait = 10, kEvKReady = 11, kEvVWait = 16, kEvVReady = 17,
-  kEvPWait = 13, kEvPReady = 14  // + 10 * Q tile
+  kEvPWait = 13, kEvPReady = 14,  // + 10 * Q tile
+  kEvSIssued = 30, kEvPVIssued = 32  // + Q tile
 };
 #ifdef EBH_PIPELINE_TRACE
 constexpr int kTraceLen = 8192;
-__device__ unsigned long long g_pipeline_trace[16][kTraceLen];
+__device__ unsigned long long g_pipeline_trace[20][kTraceLen];
 #define EBH_TRACE_COUNTER int tr_n = 0
 #define EBH_TRACE(ev, jj)                                                               \
   do {                                                                                  \
@@ -210,10 +194,6 @@ __device__ __forceinline__ TileWork decode_tile(int u, int t, const Params& p) {
   return w;
 }
 
-__device__ __forceinline__ bool in_range(const Unit& w, int t, int j) {
-  return w.valid[t] && j >= w.lo[t] && j < w.hi[t];
-}
-
 // Wait for all lanes of a warp; the outcome is made warp-uniform so that the
 // warp-collective tensor-memory instructions that follow run on all lanes or
 // none.
@@ -227,118 +207,12 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit) {
   const uint64_t t0 = globaltimer_ns();
 #pragma unroll 1
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_wait_suspend(bar, parity, 20000u)) {
     if (globaltimer_ns() - t0 > limit) {
       atomicOr(&g_attn_status_word, kStatusTimeout);
       return;
     }
   }
-}
-
-// O_t row *= alpha for this warp's 32 rows (tensor memory round trip).  The
-// caller guarantees no MMA is writing O_t (its previous P.V product was issued
-// before the S_t product the caller has waited for, and they complete in order).
-template <int D>
-__device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
-#pragma unroll 1
-  for (int c = 0; c < D / 32; ++c) {
-    uint32_t o[32];
-    tmem_ld32(tO + 32 * c, o);
-    tmem_wait_ld();
-    reg_fence32(o);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-    tmem_st32(tO + 32 * c, o);
-  }
-}
-
-// Max of n values by a tree of three-input maxima (depth log3 n).
-template <int N>
-struct TreeMax {
-  static __device__ __forceinline__ float run(float* v) {
-    constexpr int M = (N + 2) / 3;
-#pragma unroll
-    for (int i = 0; i < M; ++i) {
-      if (3 * i + 2 < N) v[i] = max3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
-      else if (3 * i + 1 < N) v[i] = fmaxf(v[3 * i], v[3 * i + 1]);
-      else v[i] = v[3 * i];
-    }
-    return TreeMax<M>::run(v);
-  }
-};
-template <>
-struct TreeMax<1> {
-  static __device__ __forceinline__ float run(float* v) { return v[0]; }
-};
-
-// Max of one row of a score tile: kMaxChains independent chains of
-// three-input maxima, or (kMaxChains == 0) a tree.
-template <int BN>
-__device__ __forceinline__ float row_max(const float* s) {
-  if constexpr (kMaxChains == 0) {
-    constexpr int M = (BN + 2) / 3;
-    float v[M];
-#pragma unroll
-    for (int i = 0; i < M; ++i) {
-      if (3 * i + 2 < BN) v[i] = max3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
-      else if (3 * i + 1 < BN) v[i] = fmaxf(s[3 * i], s[3 * i + 1]);
-      else v[i] = s[3 * i];
-    }
-    return TreeMax<M>::run(v);
-  } else {
-    constexpr int K = kMaxChains;
-    float m[K];
-#pragma unroll
-    for (int i = 0; i < K; ++i) m[i] = fmaxf(s[i], s[i + K]);
-#pragma unroll
-    for (int c = 2 * K; c < BN; c += 2 * K) {
-#pragma unroll
-      for (int i = 0; i < K; ++i) m[i] = max3(m[i], s[c + i], s[c + K + i]);
-    }
-    return TreeMax<K>::run(m);
-  }
-}
-
-// p_c = 2^(s_c * cl2 - msub) for one row of a score tile, written to tensor
-// memory as packed bf16 over the first half of the tile's S columns (those
-// scores are already in registers), 32 keys at a time.  l accumulates the
-// probabilities, lr the bf16-rounded probabilities the P.V product will use.
-// kPoly: compute one pair in kPolyEvery on the FMA pipe (tiles without masked
-// elements only: the polynomial has no -inf handling).
-template <int BN, bool kPoly>
-__device__ __forceinline__ void write_probabilities(const float* s, float cl2, float msub,
-                                                    uint32_t tS, float& l, float& lr) {
-  float la = 0.f, lb = 0.f, lc = 0.f, ld = 0.f;
-  float ra = 0.f, rb = 0.f, rc = 0.f, rd = 0.f;
-#pragma unroll
-  for (int cc = 0; cc < BN / 32; ++cc) {
-    uint32_t pk[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const int e = 32 * cc + 2 * c;
-      float x0, x1, p0, p1;
-      fma2(x0, x1, s[e], s[e + 1], cl2, cl2, -msub, -msub);
-      bool poly = false;
-      if constexpr (kPoly) poly = (c % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
-      if (poly) {
-        exp2_poly2(x0, x1, p0, p1);
-      } else {
-        p0 = ex2_approx(x0);
-        p1 = ex2_approx(x1);
-      }
-      pk[c] = pack_bf16x2(p0, p1);
-      if (c & 1) {
-        add2(lc, ld, lc, ld, p0, p1);
-        acc_bf16x2(rc, rd, pk[c]);
-      } else {
-        add2(la, lb, la, lb, p0, p1);
-        acc_bf16x2(ra, rb, pk[c]);
-      }
-    }
-    tmem_st16(tS + 16 * cc, pk);
-  }
-  l += (la + lb) + (lc + ld);
-  lr += (ra + rb) + (rc + rd);
 }
 
 template <int D, int BN>
@@ -365,9 +239,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(C::kBarQFull + t), 1);
       mbar_init(bar(C::kBarQEmpty + t), 1);
       mbar_init(bar(C::kBarSFull + t), 1);
-      mbar_init(bar(C::kBarPFull + t), kBM);
+      mbar_init(bar(C::kBarPFull + t), kSoftmaxThreads);
       mbar_init(bar(C::kBarOFull + t), 1);
-      mbar_init(bar(C::kBarOEmpty + t), kBM);
+      mbar_init(bar(C::kBarOEmpty + t), kSoftmaxThreads);
     }
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bar(C::kBarKVFull + s), 1);
@@ -398,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // on the host before launch), or the grow would wait forever.  Each role
   // runs inside the branch that set its register count, so the compiler
   // allocates each role's code under its own limit.
-  if (warp >= 8) {
+  if (warp >= kProducerWarp) {
     regs_shrink<kOtherRegs>();
     if (warp == kProducerWarp) {
       // ------------------------------------------------------------ producer
@@ -454,85 +328,109 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, BN, false);
         constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, true);
+        constexpr uint32_t kStageUnits = C::kKVTileBytes >> 4;
+        constexpr uint32_t kQTileUnits = C::kQTileBytes >> 4;
+        // Shared-memory descriptors are linear in the start address (a field
+        // in 16-byte units that cannot carry for addresses below 256 KB): keep
+        // the common high word and the three low words, add offsets per K step.
+        const uint32_t desc_hi = static_cast<uint32_t>(sdesc_sw128(0, 16, 1024) >> 32);
+        const uint32_t lo_q = static_cast<uint32_t>(sdesc_sw128(smem_addr(sQ), 16, 1024));
+        const uint32_t lo_k = static_cast<uint32_t>(sdesc_sw128(smem_addr(sKV), 16, 1024));
+        const uint32_t lo_v = static_cast<uint32_t>(sdesc_sw128(smem_addr(sKV), BN * 128, 1024));
+        auto desc = [&](uint32_t lo) -> uint64_t {
+          return (static_cast<uint64_t>(desc_hi) << 32) | lo;
+        };
         int kv_it = 0;
-        int q_cnt[kNQ] = {0, 0}, p_cnt[kNQ] = {0, 0}, o_cnt[kNQ] = {0, 0};
+        uint32_t par_q = 0, par_p = 0, par_oe = 3;  // one phase bit per Q tile
         bool ok = true;
         EBH_TRACE_COUNTER;
 
         auto issue_s = [&](int t, int kst) {
-          const uint32_t qa = smem_addr(sQ + t * C::kQTileBytes);
-          const uint32_t kb = smem_addr(sKV + kst * C::kKVTileBytes);
+          const uint32_t a0 = lo_q + t * kQTileUnits;
+          const uint32_t b0 = lo_k + kst * kStageUnits;
+          const uint32_t d = tmem + C::kColS + t * BN;
   #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint64_t a = sdesc_sw128(qa + (k / 4) * kBM * 128 + (k % 4) * 32, 16, 1024);
-            const uint64_t b = sdesc_sw128(kb + (k / 4) * BN * 128 + (k % 4) * 32, 16, 1024);
-            mma_ss(tmem + C::kColS + t * BN, a, b, idesc_s, k > 0 ? 1u : 0u);
-          }
+          for (int k = 0; k < D / 16; ++k)
+            mma_ss(d, desc(a0 + (((k / 4) * kBM * 128 + (k % 4) * 32) >> 4)),
+                   desc(b0 + (((k / 4) * BN * 128 + (k % 4) * 32) >> 4)), idesc_s,
+                   k > 0 ? 1u : 0u);
         };
         auto issue_pv = [&](int t, int vst, bool first) -> bool {
           EBH_TRACE(kEvPWait + 10 * t, 0);
-          if (!wait_bounded(bar(C::kBarPFull + t), p_cnt[t] & 1, abort_flag, limit)) return false;
+          if (!wait_bounded(bar(C::kBarPFull + t), (par_p >> t) & 1, abort_flag, limit))
+            return false;
           EBH_TRACE(kEvPReady + 10 * t, 0);
-          ++p_cnt[t];
-          if (first &&
-              !wait_bounded(bar(C::kBarOEmpty + t), (o_cnt[t] & 1) ^ 1, abort_flag, limit))
+          par_p ^= 1u << t;
+          if (first && !wait_bounded(bar(C::kBarOEmpty + t), (par_oe >> t) & 1, abort_flag, limit))
             return false;
           tc_fence_after();
-          const uint32_t vb = smem_addr(sKV + vst * C::kKVTileBytes);
+          const uint32_t b0 = lo_v + vst * kStageUnits;
+          const uint32_t d = tmem + C::kColO + t * D;
+          const uint32_t a = tmem + C::kColS + t * BN;
   #pragma unroll
-          for (int k = 0; k < BN / 16; ++k) {
-            const uint64_t b = sdesc_sw128(vb + k * 16 * 128, BN * 128, 1024);
-            mma_ts(tmem + C::kColO + t * D, tmem + C::kColS + t * BN + k * 8, b, idesc_o,
+          for (int k = 0; k < BN / 16; ++k)
+            mma_ts(d, a + k * 8, desc(b0 + ((k * 16 * 128) >> 4)), idesc_o,
                    (first && k == 0) ? 0u : 1u);
-          }
+          EBH_TRACE(kEvPVIssued + t, 0);
           return true;
         };
 
         for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-          const Unit w = decode_unit<BN>(u, p);
+          // key-block ranges of the two Q tiles (empty range: tile absent)
+          int lo0, hi0, lo1, hi1;
+          {
+            const TileWork w0 = decode_tile<BN>(u, 0, p);
+            const TileWork w1 = decode_tile<BN>(u, 1, p);
+            lo0 = w0.lo; hi0 = w0.valid ? w0.hi : w0.lo;
+            lo1 = w1.lo; hi1 = w1.valid ? w1.hi : w1.lo;
+          }
+          const bool has1 = hi1 > lo1;
+          const int ulo = has1 ? min(lo0, lo1) : lo0;
+          const int uhi = has1 ? max(hi0, hi1) : hi0;
           int pend_v = -1;  // ring stage of V_(j-1) still owed a P_1 . V product
-          for (int j = w.ulo; ok && j < w.uhi; ++j) {
+          for (int j = ulo; ok && j < uhi; ++j) {
             const int kst = kv_it % C::kStages;
             const uint32_t kph = (kv_it / C::kStages) & 1;
-            ++kv_it;
-            const int vst = kv_it % C::kStages;
-            const uint32_t vph = (kv_it / C::kStages) & 1;
-            ++kv_it;
+            const int vst = (kv_it + 1) % C::kStages;
+            const uint32_t vph = ((kv_it + 1) / C::kStages) & 1;
+            kv_it += 2;
             EBH_TRACE(kEvKWait, j);
             if (!(ok = wait_bounded(bar(C::kBarKVFull + kst), kph, abort_flag, limit))) break;
             EBH_TRACE(kEvKReady, j);
-            const bool in0 = in_range(w, 0, j), in1 = in_range(w, 1, j);
+            const bool in0 = j >= lo0 && j < hi0, in1 = j >= lo1 && j < hi1;
             if (in0) {
-              if (j == w.lo[0] &&
-                  !(ok = wait_bounded(bar(C::kBarQFull + 0), q_cnt[0] & 1, abort_flag, limit)))
+              if (j == lo0 && !(ok = wait_bounded(bar(C::kBarQFull + 0), par_q & 1, abort_flag,
+                                                  limit)))
                 break;
               tc_fence_after();
               issue_s(0, kst);
+              EBH_TRACE(kEvSIssued + 0, j);
               mma_commit(bar(C::kBarSFull + 0));
-              if (j == w.hi[0] - 1) mma_commit(bar(C::kBarQEmpty + 0));
+              if (j == hi0 - 1) mma_commit(bar(C::kBarQEmpty + 0));
             }
             if (pend_v >= 0) {
-              if (!(ok = issue_pv(1, pend_v, j - 1 == w.lo[1]))) break;
+              if (!(ok = issue_pv(1, pend_v, j - 1 == lo1))) break;
               mma_commit(bar(C::kBarKVEmpty + pend_v));
-              if (j - 1 == w.hi[1] - 1) mma_commit(bar(C::kBarOFull + 1));
+              if (j - 1 == hi1 - 1) mma_commit(bar(C::kBarOFull + 1));
               pend_v = -1;
             }
             if (in1) {
-              if (j == w.lo[1] &&
-                  !(ok = wait_bounded(bar(C::kBarQFull + 1), q_cnt[1] & 1, abort_flag, limit)))
+              if (j == lo1 && !(ok = wait_bounded(bar(C::kBarQFull + 1), (par_q >> 1) & 1,
+                                                  abort_flag, limit)))
                 break;
               tc_fence_after();
               issue_s(1, kst);
+              EBH_TRACE(kEvSIssued + 1, j);
               mma_commit(bar(C::kBarSFull + 1));
-              if (j == w.hi[1] - 1) mma_commit(bar(C::kBarQEmpty + 1));
+              if (j == hi1 - 1) mma_commit(bar(C::kBarQEmpty + 1));
             }
             mma_commit(bar(C::kBarKVEmpty + kst));  // K_j no longer needed
             EBH_TRACE(kEvVWait, j);
             if (!(ok = wait_bounded(bar(C::kBarKVFull + vst), vph, abort_flag, limit))) break;
             EBH_TRACE(kEvVReady, j);
             if (in0) {
-              if (!(ok = issue_pv(0, vst, j == w.lo[0]))) break;
-              if (j == w.hi[0] - 1) mma_commit(bar(C::kBarOFull + 0));
+              if (!(ok = issue_pv(0, vst, j == lo0))) break;
+              if (j == hi0 - 1) mma_commit(bar(C::kBarOFull + 0));
             }
             if (in1) {
               pend_v = vst;
@@ -541,20 +439,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (ok && pend_v >= 0) {
-            const int j = w.uhi;
-            if ((ok = issue_pv(1, pend_v, j - 1 == w.lo[1]))) {
+            if ((ok = issue_pv(1, pend_v, uhi - 1 == lo1))) {
               mma_commit(bar(C::kBarKVEmpty + pend_v));
-              if (j - 1 == w.hi[1] - 1) mma_commit(bar(C::kBarOFull + 1));
+              if (uhi - 1 == hi1 - 1) mma_commit(bar(C::kBarOFull + 1));
             }
           }
-          if (w.valid[0]) {
-            ++q_cnt[0];
-            ++o_cnt[0];
-          }
-          if (w.valid[1]) {
-            ++q_cnt[1];
-            ++o_cnt[1];
-          }
+          // Q tiles and O accumulators used by this unit move to their next phase
+          const uint32_t used = (hi0 > lo0 ? 1u : 0u) | (has1 ? 2u : 0u);
+          par_q ^= used;
+          par_oe ^= used;
         }
         // No MMA may still be writing tensor memory when it is freed.
         mma_commit(bar(C::kBarDrain));
@@ -563,13 +456,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
+    // Eight warps per Q tile, two per tensor-memory sub-partition (lanes
+    // 32q..32q+15 and 32q+16..32q+31).  Four threads share a row: lane l holds
+    // rows l/4 and l/4 + 8 of its warp's 16, and the key columns 8m + 2(l%4)
+    // and 8m + 2(l%4) + 1 of every group of eight.
     regs_grow<kSoftmaxRegs>();
-    const int t = warp / 4;
-    const int wq = warp % 4;                 // this warp's 32-lane slice of tensor memory
-    const int r = threadIdx.x % kBM;         // query row within the Q tile
-    const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
-    const uint32_t tS = tmem + lane_base + C::kColS + t * BN;
-    const uint32_t tO = tmem + lane_base + C::kColO + t * D;
+    const int t = warp / kSoftmaxWarps;
+    const int wl = warp % kSoftmaxWarps;
+    const int lbase = 32 * (warp % 4) + 16 * (wl / 4);  // first row (= lane) of this warp
+    const int t0 = lane % 4;
+    const int ra = lbase + lane / 4;                   // the thread's rows in the Q tile
+    const int rb = ra + 8;
+    const uint32_t lane_addr = static_cast<uint32_t>(lbase) << 16;
+    const uint32_t tS = tmem + lane_addr + C::kColS + t * BN;
+    const uint32_t tO = tmem + lane_addr + C::kColO + t * D;
     const float cl2 = p.scale_log2;
     int s_cnt = 0, o_cnt = 0;
     bool ok = true;
@@ -578,10 +478,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
       const TileWork w = decode_tile<BN>(u, t, p);
       if (!w.valid) continue;
-      const int row = w.q_first + r;
-      float m_used = -INFINITY;  // running max, log2 units
-      float l = 0.f;             // running sum of the probabilities against m_used
-      float lr = 0.f;            // the same sum over the bf16-rounded probabilities
+      const int row_a = w.q_first + ra, row_b = w.q_first + rb;
+      // per row: running max (log2 units), sums of the probabilities against
+      // it (two partial accumulators each) and of their bf16 roundings
+      float m_a = -INFINITY, m_b = -INFINITY;
+      float la0 = 0.f, la1 = 0.f, lb0 = 0.f, lb1 = 0.f;
+      float ra0 = 0.f, ra1 = 0.f, rb0 = 0.f, rb1 = 0.f;
 
       for (int j = w.lo; j < w.hi; ++j) {
         EBH_TRACE(kEvSWait, j);
@@ -589,71 +491,118 @@ __global__ void __launch_bounds__(kThreads, 1)
         EBH_TRACE(kEvSReady, j);
         ++s_cnt;
         tc_fence_after();
-        uint32_t sr[BN];
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + 32 * c, sr + 32 * c);
+        uint32_t sr[BN / 2];
+        if constexpr (BN == 128) {
+          tmem_ld_16x256b_x16(tS, sr);
+        } else {
+          tmem_ld_16x256b_x8(tS, sr);
+        }
         tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) reg_fence32(sr + 32 * c);
+        if constexpr (BN == 128) {
+          reg_fence64(sr);
+        } else {
+          reg_fence32(sr);
+        }
         float* s = reinterpret_cast<float*>(sr);
         EBH_TRACE(kEvSLoaded, j);
 
         const bool full =
             kv_tile_class(p.L, w.q_first, w.q_last, j, p.mask_kind, p.window, BN) == kTileFull;
         if (!full) {
-          int c_lo, c_hi;
-          row_allowed_cols(p.L, row, j, p.mask_kind, p.window, BN, c_lo, c_hi);
+          int a_lo, a_hi, b_lo, b_hi;
+          row_allowed_cols(p.L, row_a, j, p.mask_kind, p.window, BN, a_lo, a_hi);
+          row_allowed_cols(p.L, row_b, j, p.mask_kind, p.window, BN, b_lo, b_hi);
 #pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c < c_lo || c >= c_hi) s[c] = -INFINITY;
+          for (int m = 0; m < BN / 8; ++m) {
+            const int c = 8 * m + 2 * t0;
+            if (c < a_lo || c >= a_hi) s[4 * m] = -INFINITY;
+            if (c + 1 < a_lo || c + 1 >= a_hi) s[4 * m + 1] = -INFINITY;
+            if (c < b_lo || c >= b_hi) s[4 * m + 2] = -INFINITY;
+            if (c + 1 < b_lo || c + 1 >= b_hi) s[4 * m + 3] = -INFINITY;
+          }
         }
         EBH_TRACE(kEvMasked, j);
-        const float m_tile = row_max<BN>(s) * cl2;
-        if (!kSpeculate || m_used == -INFINITY) {
-          float alpha = 1.f;
-          bool rescale = false;
-          if (m_used == -INFINITY) {
-            // nothing accumulated for this row yet (l == 0 and its O row is 0)
-            m_used = m_tile;
-          } else if (m_tile > m_used + kRescaleThreshold) {
-            alpha = ex2_approx(m_used - m_tile);
-            l *= alpha;
-            lr *= alpha;
-            m_used = m_tile;
-            rescale = true;
-          }
-          if (__any_sync(0xffffffffu, rescale)) rescale_o_row<D>(tO, alpha);
-          const float msub = m_used == -INFINITY ? 0.f : m_used;
-          EBH_TRACE(kEvMaxDone, j);
-          if (full) {
-            write_probabilities<BN, (kPolyEvery > 0)>(s, cl2, msub, tS, l, lr);
+        // row maxima: this thread's 2 x (BN / 4) scores, then across the four
+        // threads of each row
+        float xa0 = s[0], xa1 = s[1], xb0 = s[2], xb1 = s[3];
+#pragma unroll
+        for (int m = 1; m < BN / 8; m += 2) {
+          if (m + 1 < BN / 8) {
+            xa0 = max3(xa0, s[4 * m], s[4 * m + 4]);
+            xa1 = max3(xa1, s[4 * m + 1], s[4 * m + 5]);
+            xb0 = max3(xb0, s[4 * m + 2], s[4 * m + 6]);
+            xb1 = max3(xb1, s[4 * m + 3], s[4 * m + 7]);
           } else {
-            write_probabilities<BN, false>(s, cl2, msub, tS, l, lr);
+            xa0 = fmaxf(xa0, s[4 * m]);
+            xa1 = fmaxf(xa1, s[4 * m + 1]);
+            xb0 = fmaxf(xb0, s[4 * m + 2]);
+            xb1 = fmaxf(xb1, s[4 * m + 3]);
           }
-        } else {
-          // Speculate that the stale reference m_used still holds (the tile
-          // max exceeds it by at most the threshold), so the exponentials do
-          // not wait for the max; if it does not hold for some row, redo the
-          // tile against the new max and rescale that row of O.
-          const float l0 = l, lr0 = lr;
-          EBH_TRACE(kEvMaxDone, j);
-          if (full) {
-            write_probabilities<BN, (kPolyEvery > 0)>(s, cl2, m_used, tS, l, lr);
-          } else {
-            write_probabilities<BN, false>(s, cl2, m_used, tS, l, lr);
+        }
+        float mta = fmaxf(xa0, xa1), mtb = fmaxf(xb0, xb1);
+        mta = fmaxf(mta, __shfl_xor_sync(0xffffffffu, mta, 1));
+        mtb = fmaxf(mtb, __shfl_xor_sync(0xffffffffu, mtb, 1));
+        mta = fmaxf(mta, __shfl_xor_sync(0xffffffffu, mta, 2));
+        mtb = fmaxf(mtb, __shfl_xor_sync(0xffffffffu, mtb, 2));
+        mta *= cl2;
+        mtb *= cl2;
+        // lazy rescale, per row (the four threads of a row decide alike)
+        float alpha_a = 1.f, alpha_b = 1.f;
+        bool rescale = false;
+        if (m_a == -INFINITY) {
+          m_a = mta;  // nothing accumulated for this row yet
+        } else if (mta > m_a + kRescaleThreshold) {
+          alpha_a = ex2_approx(m_a - mta);
+          m_a = mta;
+          rescale = true;
+        }
+        if (m_b == -INFINITY) {
+          m_b = mtb;
+        } else if (mtb > m_b + kRescaleThreshold) {
+          alpha_b = ex2_approx(m_b - mtb);
+          m_b = mtb;
+          rescale = true;
+        }
+        if (__any_sync(0xffffffffu, rescale)) {
+          la0 *= alpha_a; la1 *= alpha_a; ra0 *= alpha_a; ra1 *= alpha_a;
+          lb0 *= alpha_b; lb1 *= alpha_b; rb0 *= alpha_b; rb1 *= alpha_b;
+          // O_t's previous product is complete (it was issued before S_t(j))
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[16];
+            tmem_ld_16x256b_x4(tO + 32 * c, o);
+            tmem_wait_ld();
+            reg_fence16(o);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              o[i] = __float_as_uint(__uint_as_float(o[i]) * ((i & 2) ? alpha_b : alpha_a));
+            tmem_st_16x256b_x4(tO + 32 * c, o);
           }
-          const bool redo = m_tile > m_used + kRescaleThreshold;
-          if (__any_sync(0xffffffffu, redo)) {
-            float alpha = 1.f;
-            if (redo) {
-              alpha = ex2_approx(m_used - m_tile);
-              m_used = m_tile;
-            }
-            l = l0 * alpha;
-            lr = lr0 * alpha;
-            rescale_o_row<D>(tO, alpha);
-            write_probabilities<BN, false>(s, cl2, m_used, tS, l, lr);
+        }
+        const float sa = m_a == -INFINITY ? 0.f : m_a;
+        const float sb = m_b == -INFINITY ? 0.f : m_b;
+        EBH_TRACE(kEvMaxDone, j);
+        // probabilities -> packed bf16 over the first half of S_t, four
+        // column groups (16 packed columns) per store
+#pragma unroll
+        for (int ch = 0; ch < BN / 32; ++ch) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int mm = 0; mm < 4; ++mm) {
+            const int m = 4 * ch + mm;
+            float x0, x1, x2, x3;
+            fma2(x0, x1, s[4 * m], s[4 * m + 1], cl2, cl2, -sa, -sa);
+            fma2(x2, x3, s[4 * m + 2], s[4 * m + 3], cl2, cl2, -sb, -sb);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+            pk[2 * mm] = pack_bf16x2(p0, p1);
+            pk[2 * mm + 1] = pack_bf16x2(p2, p3);
+            add2(la0, la1, la0, la1, p0, p1);
+            add2(lb0, lb1, lb0, lb1, p2, p3);
+            acc_bf16x2(ra0, ra1, pk[2 * mm]);
+            acc_bf16x2(rb0, rb1, pk[2 * mm + 1]);
           }
+          tmem_st_16x128b_x4(tS + 16 * ch, pk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -662,37 +611,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
 
-      // ---- epilogue: O / l -> bf16, LSE = ln 2 * (m + log2 l)
+      // ---- epilogue: O / lr -> bf16, LSE = ln 2 * (m + log2 l)
       EBH_TRACE(kEvEpilogue, 0);
       if (!(ok = warp_wait(bar(C::kBarOFull + t), o_cnt & 1, abort_flag, limit))) break;
       ++o_cnt;
       tc_fence_after();
+      float l_a = la0 + la1, l_b = lb0 + lb1, lr_a = ra0 + ra1, lr_b = rb0 + rb1;
+#pragma unroll
+      for (int x = 1; x <= 2; x <<= 1) {
+        l_a += __shfl_xor_sync(0xffffffffu, l_a, x);
+        l_b += __shfl_xor_sync(0xffffffffu, l_b, x);
+        lr_a += __shfl_xor_sync(0xffffffffu, lr_a, x);
+        lr_b += __shfl_xor_sync(0xffffffffu, lr_b, x);
+      }
       // O is divided by the sum of exactly the (bf16) weights that multiplied
       // V, so the weights sum to one; LSE uses the unrounded sum.
-      const float inv_l = lr > 0.f ? 1.f / lr : 0.f;
-      const bool row_ok = row < p.L;
-      const size_t row_off = (static_cast<size_t>(w.bh) * p.L + (row_ok ? row : 0)) * D;
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + row_off);
+      const float inv_a = lr_a > 0.f ? 1.f / lr_a : 0.f;
+      const float inv_b = lr_b > 0.f ? 1.f / lr_b : 0.f;
+      const bool ok_a = row_a < p.L, ok_b = row_b < p.L;
+      uint32_t* dst_a = reinterpret_cast<uint32_t*>(
+          static_cast<uint16_t*>(p.out) +
+          (static_cast<size_t>(w.bh) * p.L + (ok_a ? row_a : 0)) * D);
+      uint32_t* dst_b = reinterpret_cast<uint32_t*>(
+          static_cast<uint16_t*>(p.out) +
+          (static_cast<size_t>(w.bh) * p.L + (ok_b ? row_b : 0)) * D);
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + 32 * c, o);
+        uint32_t o[16];
+        tmem_ld_16x256b_x4(tO + 32 * c, o);
         tmem_wait_ld();
-        reg_fence32(o);
-        uint32_t pk[16];
+        reg_fence16(o);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
-                              __uint_as_float(o[2 * i + 1]) * inv_l);
-        if (row_ok) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[c * 4 + i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        for (int mm = 0; mm < 4; ++mm) {
+          const int col2 = (32 * c + 8 * mm + 2 * t0) / 2;  // pair index in the row
+          const uint32_t va = pack_bf16x2(__uint_as_float(o[4 * mm]) * inv_a,
+                                          __uint_as_float(o[4 * mm + 1]) * inv_a);
+          const uint32_t vb = pack_bf16x2(__uint_as_float(o[4 * mm + 2]) * inv_b,
+                                          __uint_as_float(o[4 * mm + 3]) * inv_b);
+          if (ok_a) dst_a[col2] = va;
+          if (ok_b) dst_b[col2] = vb;
         }
       }
-      if (row_ok && p.lse != nullptr) {
-        const float lse = l > 0.f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
-        p.lse[static_cast<size_t>(w.bh) * p.L + row] = lse;
+      if (t0 == 0 && p.lse != nullptr) {
+        if (ok_a)
+          p.lse[static_cast<size_t>(w.bh) * p.L + row_a] =
+              l_a > 0.f ? (m_a + log2f(l_a)) * 0.69314718055994531f : -INFINITY;
+        if (ok_b)
+          p.lse[static_cast<size_t>(w.bh) * p.L + row_b] =
+              l_b > 0.f ? (m_b + log2f(l_b)) * 0.69314718055994531f : -INFINITY;
       }
       tc_fence_before();
       EBH_TRACE(kEvEpilogueDone, 0);
@@ -883,7 +849,7 @@ extern "C" __attribute__((visibility("default"))) int attn_pipeline_trace_read(
       cudaMemcpyFromSymbol(host, ebh::g_pipeline_trace, sizeof(ebh::g_pipeline_trace)));
 }
 extern "C" __attribute__((visibility("default"))) int attn_pipeline_trace_clear() {
-  static unsigned long long zero[16][ebh::kTraceLen];
+  static unsigned long long zero[20][ebh::kTraceLen];
   return static_cast<int>(cudaMemcpyToSymbol(ebh::g_pipeline_trace, zero, sizeof(zero)));
 }
 #endif
