@@ -34,7 +34,7 @@ ATTN_DTYPE_F32 = 1
 # Every entry point declared in include/attn.h.
 EXPORTED = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ex", "attn_strerror", "attn_last_cuda_error",
             "attn_device_status", "attn_selftest_wait_timeout", "attn_kv_tile_range",
-            "attn_kv_tile_class", "attn_abi_version")
+            "attn_kv_tile_class", "attn_kv_full_range", "attn_abi_version")
 
 
 class AttnParams(ctypes.Structure):
@@ -93,6 +93,8 @@ def _load():
             lib.attn_kv_tile_range.argtypes = [i, i, i, i, i, i, ctypes.POINTER(i),
                                                ctypes.POINTER(i)]
             lib.attn_kv_tile_class.argtypes = [i, i, i, i, i, i, i]
+            lib.attn_kv_full_range.argtypes = [i, i, i, i, i, i, ctypes.POINTER(i),
+                                               ctypes.POINTER(i)]
             lib.attn_abi_version.argtypes = []
             for name in EXPORTED:
                 if name != "attn_strerror":
@@ -174,6 +176,15 @@ def kv_tile_range(L, q_first, q_last, mask="none", window=0, block_n=128):
                                     ctypes.byref(lo), ctypes.byref(hi))
     if st != ATTN_OK:
         raise AttnError(st, "attn_kv_tile_range")
+    return lo.value, hi.value
+
+
+def kv_full_range(L, q_first, q_last, mask="none", window=0, block_n=128):
+    lo, hi = ctypes.c_int(), ctypes.c_int()
+    st = _load().attn_kv_full_range(L, q_first, q_last, MASK_KINDS[mask], window, block_n,
+                                    ctypes.byref(lo), ctypes.byref(hi))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_kv_full_range")
     return lo.value, hi.value
 
 

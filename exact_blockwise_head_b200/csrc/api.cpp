@@ -215,6 +215,16 @@ int attn_kv_tile_class(int L, int q_first, int q_last, int j, int mask_kind, int
   return ebh::kv_tile_class(L, q_first, q_last, j, mask_kind, window, block_n);
 }
 
+int attn_kv_full_range(int L, int q_first, int q_last, int mask_kind, int window, int block_n,
+                       int* lo, int* hi) {
+  if (!lo || !hi || L <= 0 || block_n <= 0 || q_first < 0 || q_last < q_first || q_last >= L)
+    return ATTN_ERR_INVALID;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_WINDOW) return ATTN_ERR_INVALID;
+  if (mask_kind == ATTN_MASK_WINDOW && window < 0) return ATTN_ERR_INVALID;
+  ebh::kv_full_range(L, q_first, q_last, mask_kind, window, block_n, *lo, *hi);
+  return ATTN_OK;
+}
+
 int attn_abi_version(void) { return ATTN_ABI_VERSION; }
 
 }  // extern "C"

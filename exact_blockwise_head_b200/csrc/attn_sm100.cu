@@ -58,6 +58,14 @@ constexpr int kSoftmaxRegs = 104;
 constexpr int kOtherRegs = 64;
 static_assert(kSoftmaxRegs * kNQ * kSoftmaxThreads + kOtherRegs * 128 <= kLaunchRegs * kThreads,
               "register split exceeds the launch allocation");
+// Share of the exponentials computed on the FMA pipe by a polynomial instead of
+// the MUFU pipe (on tiles without masked elements): one column group of eight
+// in kPolyEvery (0 = none).  The MUFU work per tile otherwise equals the
+// tensor-core work the softmax has to hide behind.
+#ifndef EBH_POLY_EVERY
+#define EBH_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = EBH_POLY_EVERY;
 // Lazy rescale: keep the stale max until the row max exceeds it by more than
 // 2^8 (probabilities then stay <= 256, far inside fp32/bf16 range).
 constexpr float kRescaleThreshold = 8.0f;
@@ -471,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tS = tmem + lane_addr + C::kColS + t * BN;
     const uint32_t tO = tmem + lane_addr + C::kColO + t * D;
     const float cl2 = p.scale_log2;
-    int s_cnt = 0, o_cnt = 0;
+    uint32_t phase = 0;  // bit 0: S_full parity, bit 1: O_full parity
     bool ok = true;
     EBH_TRACE_COUNTER;
 
@@ -479,17 +487,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const TileWork w = decode_tile<BN>(u, t, p);
       if (!w.valid) continue;
       const int row_a = w.q_first + ra, row_b = w.q_first + rb;
-      // per row: running max (log2 units), sums of the probabilities against
-      // it (two partial accumulators each) and of their bf16 roundings
+      int full_lo, full_hi;  // key blocks that need no element mask
+      kv_full_range(p.L, w.q_first, w.q_last, p.mask_kind, p.window, BN, full_lo, full_hi);
+      // per row: running max (log2 units), sum of the probabilities against
+      // it and sum of their bf16 roundings
       float m_a = -INFINITY, m_b = -INFINITY;
-      float la0 = 0.f, la1 = 0.f, lb0 = 0.f, lb1 = 0.f;
-      float ra0 = 0.f, ra1 = 0.f, rb0 = 0.f, rb1 = 0.f;
+      float l_a = 0.f, l_b = 0.f, lr_a = 0.f, lr_b = 0.f;
 
       for (int j = w.lo; j < w.hi; ++j) {
         EBH_TRACE(kEvSWait, j);
-        if (!(ok = warp_wait(bar(C::kBarSFull + t), s_cnt & 1, abort_flag, limit))) break;
+        if (!(ok = warp_wait(bar(C::kBarSFull + t), phase & 1, abort_flag, limit))) break;
         EBH_TRACE(kEvSReady, j);
-        ++s_cnt;
+        phase ^= 1;
         tc_fence_after();
         uint32_t sr[BN / 2];
         if constexpr (BN == 128) {
@@ -504,10 +513,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           reg_fence32(sr);
         }
         float* s = reinterpret_cast<float*>(sr);
-        EBH_TRACE(kEvSLoaded, j);
+#ifdef EBH_PIPELINE_TRACE
+        {  // profiling builds: stamp only once the loaded scores are really in registers
+          const uint32_t probe = __shfl_sync(0xffffffffu, sr[BN / 2 - 1] ^ sr[0], 0);
+          EBH_TRACE(kEvSLoaded, j + (probe == 0x7fc00001u ? 1 : 0));
+        }
+#endif
 
-        const bool full =
-            kv_tile_class(p.L, w.q_first, w.q_last, j, p.mask_kind, p.window, BN) == kTileFull;
+        const bool full = j >= full_lo && j < full_hi;
         if (!full) {
           int a_lo, a_hi, b_lo, b_hi;
           row_allowed_cols(p.L, row_a, j, p.mask_kind, p.window, BN, a_lo, a_hi);
@@ -564,8 +577,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           rescale = true;
         }
         if (__any_sync(0xffffffffu, rescale)) {
-          la0 *= alpha_a; la1 *= alpha_a; ra0 *= alpha_a; ra1 *= alpha_a;
-          lb0 *= alpha_b; lb1 *= alpha_b; rb0 *= alpha_b; rb1 *= alpha_b;
+          l_a *= alpha_a; lr_a *= alpha_a;
+          l_b *= alpha_b; lr_b *= alpha_b;
           // O_t's previous product is complete (it was issued before S_t(j))
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
@@ -590,17 +603,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int mm = 0; mm < 4; ++mm) {
             const int m = 4 * ch + mm;
-            float x0, x1, x2, x3;
+            float x0, x1, x2, x3, p0, p1, p2, p3;
             fma2(x0, x1, s[4 * m], s[4 * m + 1], cl2, cl2, -sa, -sa);
             fma2(x2, x3, s[4 * m + 2], s[4 * m + 3], cl2, cl2, -sb, -sb);
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-            const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+            if (kPolyEvery > 0 && full && (m % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+              // this group's exponentials on the FMA pipe (no -inf here: the
+              // tile has no masked element)
+              exp2_poly2(x0, x1, p0, p1);
+              exp2_poly2(x2, x3, p2, p3);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+              p2 = ex2_approx(x2);
+              p3 = ex2_approx(x3);
+            }
             pk[2 * mm] = pack_bf16x2(p0, p1);
             pk[2 * mm + 1] = pack_bf16x2(p2, p3);
-            add2(la0, la1, la0, la1, p0, p1);
-            add2(lb0, lb1, lb0, lb1, p2, p3);
-            acc_bf16x2(ra0, ra1, pk[2 * mm]);
-            acc_bf16x2(rb0, rb1, pk[2 * mm + 1]);
+            add2(l_a, l_b, l_a, l_b, p0, p2);
+            add2(l_a, l_b, l_a, l_b, p1, p3);
+            acc_bf16x2_sum(lr_a, pk[2 * mm]);
+            acc_bf16x2_sum(lr_b, pk[2 * mm + 1]);
           }
           tmem_st_16x128b_x4(tS + 16 * ch, pk);
         }
@@ -613,10 +635,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // ---- epilogue: O / lr -> bf16, LSE = ln 2 * (m + log2 l)
       EBH_TRACE(kEvEpilogue, 0);
-      if (!(ok = warp_wait(bar(C::kBarOFull + t), o_cnt & 1, abort_flag, limit))) break;
-      ++o_cnt;
+      if (!(ok = warp_wait(bar(C::kBarOFull + t), (phase >> 1) & 1, abort_flag, limit))) break;
+      phase ^= 2;
       tc_fence_after();
-      float l_a = la0 + la1, l_b = lb0 + lb1, lr_a = ra0 + ra1, lr_b = rb0 + rb1;
 #pragma unroll
       for (int x = 1; x <= 2; x <<= 1) {
         l_a += __shfl_xor_sync(0xffffffffu, l_a, x);

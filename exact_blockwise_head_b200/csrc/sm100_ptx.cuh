@@ -395,6 +395,13 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
+// a += both bf16 halves of `pk`, each widened exactly.
+__device__ __forceinline__ void acc_bf16x2_sum(float& a, uint32_t pk) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %0, hi, %0;\n\t}"
+      : "+f"(a)
+      : "r"(pk));
+}
 // (a, b) += the two bf16 halves of `pk` (low half to a), each widened exactly.
 __device__ __forceinline__ void acc_bf16x2(float& a, float& b, uint32_t pk) {
   asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"

@@ -59,6 +59,28 @@ EBH_HD int kv_tile_class(int L, int q_first, int q_last, int j, int mask_kind,
   return k1 < L ? kTileFull : kTilePartial;
 }
 
+// Key blocks [flo, fhi) in which every pair of rows [q_first, q_last] and
+// keys is allowed and every key is < L (the FULL blocks of kv_tile_class, which
+// always form one contiguous run; flo == fhi when there are none).
+EBH_HD void kv_full_range(int L, int q_first, int q_last, int mask_kind, int window, int bn,
+                          int& flo, int& fhi) {
+  long long lo = 0, hi = L / bn;  // blocks entirely below L
+  if (mask_kind == kMaskCausal) {
+    // (j + 1) bn - 1 <= q_first
+    const long long h = ((long long)q_first + 1) / bn;
+    if (h < hi) hi = h;
+  } else if (mask_kind == kMaskWindow) {
+    // q_last - j bn <= w  and  (j + 1) bn - 1 - q_first <= w
+    const long long a = (long long)q_last - window;
+    if (a > 0) lo = (a + bn - 1) / bn;
+    const long long h = ((long long)q_first + window + 1) / bn;
+    if (h < hi) hi = h;
+  }
+  if (hi < lo) hi = lo;
+  flo = (int)lo;
+  fhi = (int)hi;
+}
+
 // Allowed key columns [c_lo, c_hi) of row i inside key block j (block of bn
 // keys starting at j*bn), clipped to the keys < L.
 EBH_HD void row_allowed_cols(int L, int i, int j, int mask_kind, int window,

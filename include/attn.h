@@ -161,6 +161,10 @@ ATTN_API int attn_kv_tile_range(int L, int q_first, int q_last, int mask_kind, i
                        int block_n, int* lo, int* hi);
 ATTN_API int attn_kv_tile_class(int L, int q_first, int q_last, int j, int mask_kind,
                        int window, int block_n);
+/* The FULL blocks always form one contiguous run [lo, hi) (lo == hi: none);
+ * the kernels test j against it instead of classifying every block. */
+ATTN_API int attn_kv_full_range(int L, int q_first, int q_last, int mask_kind, int window,
+                                int block_n, int* lo, int* hi);
 
 /* ATTN_ABI_VERSION of the loaded library. */
 ATTN_API int attn_abi_version(void);

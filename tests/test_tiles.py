@@ -47,6 +47,9 @@ def test_range_and_class_match_dense_mask(L, mask, window):
                 assert cls == expect, (L, mask, window, bn, q_first, j, cls, expect)
                 # tiles outside [lo, hi) hold no allowed pair; inside, at least one
                 assert (lo <= j < hi) == (expect != 0), (L, mask, window, bn, q_first, j)
+                # the FULL blocks are exactly the contiguous run [flo, fhi)
+                flo, fhi = ebh.kv_full_range(L, q_first, q_last, mask, window, bn)
+                assert (flo <= j < fhi) == (expect == 2), (L, mask, window, bn, q_first, j)
 
 
 def test_bad_tile_arguments():
