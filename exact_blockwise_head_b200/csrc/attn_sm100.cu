@@ -58,14 +58,6 @@ constexpr int kSoftmaxRegs = 104;
 constexpr int kOtherRegs = 64;
 static_assert(kSoftmaxRegs * kNQ * kSoftmaxThreads + kOtherRegs * 128 <= kLaunchRegs * kThreads,
               "register split exceeds the launch allocation");
-// Share of the exponentials computed on the FMA pipe by a polynomial instead of
-// the MUFU pipe (on tiles without masked elements): one column group of eight
-// in kPolyEvery (0 = none).  The MUFU work per tile otherwise equals the
-// tensor-core work the softmax has to hide behind.
-#ifndef EBH_POLY_EVERY
-#define EBH_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = EBH_POLY_EVERY;
 // Lazy rescale: keep the stale max until the row max exceeds it by more than
 // 2^8 (probabilities then stay <= 256, far inside fp32/bf16 range).
 constexpr float kRescaleThreshold = 8.0f;
@@ -220,6 +212,116 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
       atomicOr(&g_attn_status_word, kStatusTimeout);
       return;
     }
+  }
+}
+
+// ---- softmax helpers (four threads per row, two rows per thread; see the
+// softmax section of the kernel for the register layout)
+
+// Load / fence half a score row block: BN/2 keys = BN/16 column groups.
+template <int BN>
+__device__ __forceinline__ void tmem_ld_half(uint32_t taddr, uint32_t* r) {
+  if constexpr (BN == 128) {
+    tmem_ld_16x256b_x8(taddr, r);
+  } else {
+    tmem_ld_16x256b_x4(taddr, r);
+  }
+}
+template <int BN>
+__device__ __forceinline__ void reg_fence_half(uint32_t* r) {
+  if constexpr (BN == 128) {
+    reg_fence32(r);
+  } else {
+    reg_fence16(r);
+  }
+}
+
+// -inf for the keys outside each row's allowed columns, groups [G0, G1).
+template <int G0, int G1>
+__device__ __forceinline__ void mask_groups(float* s, int t0, int a_lo, int a_hi, int b_lo,
+                                            int b_hi) {
+#pragma unroll
+  for (int m = G0; m < G1; ++m) {
+    const int c = 8 * m + 2 * t0;
+    if (c < a_lo || c >= a_hi) s[4 * m] = -INFINITY;
+    if (c + 1 < a_lo || c + 1 >= a_hi) s[4 * m + 1] = -INFINITY;
+    if (c < b_lo || c >= b_hi) s[4 * m + 2] = -INFINITY;
+    if (c + 1 < b_lo || c + 1 >= b_hi) s[4 * m + 3] = -INFINITY;
+  }
+}
+
+// Row maxima of the thread's two rows over the whole block, then across the
+// four threads that share each row.
+template <int BN>
+__device__ __forceinline__ void row_max_pair(const float* s, float& mta, float& mtb) {
+  float xa0 = s[0], xa1 = s[1], xb0 = s[2], xb1 = s[3];
+#pragma unroll
+  for (int m = 1; m < BN / 8; m += 2) {
+    if (m + 1 < BN / 8) {
+      xa0 = max3(xa0, s[4 * m], s[4 * m + 4]);
+      xa1 = max3(xa1, s[4 * m + 1], s[4 * m + 5]);
+      xb0 = max3(xb0, s[4 * m + 2], s[4 * m + 6]);
+      xb1 = max3(xb1, s[4 * m + 3], s[4 * m + 7]);
+    } else {
+      xa0 = fmaxf(xa0, s[4 * m]);
+      xa1 = fmaxf(xa1, s[4 * m + 1]);
+      xb0 = fmaxf(xb0, s[4 * m + 2]);
+      xb1 = fmaxf(xb1, s[4 * m + 3]);
+    }
+  }
+  mta = fmaxf(xa0, xa1);
+  mtb = fmaxf(xb0, xb1);
+  mta = fmaxf(mta, __shfl_xor_sync(0xffffffffu, mta, 1));
+  mtb = fmaxf(mtb, __shfl_xor_sync(0xffffffffu, mtb, 1));
+  mta = fmaxf(mta, __shfl_xor_sync(0xffffffffu, mta, 2));
+  mtb = fmaxf(mtb, __shfl_xor_sync(0xffffffffu, mtb, 2));
+}
+
+// p = 2^(s cl2 - m) for column groups [G0, G1) (multiples of 4), packed to bf16
+// and written over the first half of S_t (group m -> packed column 4m + t0);
+// l += p, lr += bf16(p), per row.
+template <int G0, int G1>
+__device__ __forceinline__ void probabilities(const float* s, float cl2, float ma, float mb,
+                                              uint32_t tS, float& l_a, float& l_b, float& lr_a,
+                                              float& lr_b) {
+#pragma unroll
+  for (int ch = G0 / 4; ch < G1 / 4; ++ch) {
+    uint32_t pk[8];
+#pragma unroll
+    for (int mm = 0; mm < 4; ++mm) {
+      const int m = 4 * ch + mm;
+      float x0, x1, x2, x3;
+      fma2(x0, x1, s[4 * m], s[4 * m + 1], cl2, cl2, -ma, -ma);
+      fma2(x2, x3, s[4 * m + 2], s[4 * m + 3], cl2, cl2, -mb, -mb);
+      const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+      const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+      pk[2 * mm] = pack_bf16x2(p0, p1);
+      pk[2 * mm + 1] = pack_bf16x2(p2, p3);
+      add2(l_a, l_b, l_a, l_b, p0, p2);
+      add2(l_a, l_b, l_a, l_b, p1, p3);
+      acc_bf16x2_sum(lr_a, pk[2 * mm]);
+      acc_bf16x2_sum(lr_b, pk[2 * mm + 1]);
+    }
+    tmem_st_16x128b_x4(tS + 16 * ch, pk);
+  }
+}
+
+// O rows *= alpha (alpha_a for the thread's first row, alpha_b for its
+// second), all D columns, through tensor memory.  The caller guarantees no MMA
+// is writing O_t (its previous P.V product was issued before the S_t product
+// the caller has waited for, and tcgen05 MMAs complete in order).
+template <int D>
+__device__ __forceinline__ void rescale_o_rows(uint32_t tO, float alpha_a, float alpha_b) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[16];
+    tmem_ld_16x256b_x4(tO + 32 * c, o);
+    tmem_wait_ld();
+    reg_fence16(o);
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      o[i] = __float_as_uint(__uint_as_float(o[i]) * ((i & 2) ? alpha_b : alpha_a));
+    tmem_st_16x256b_x4(tO + 32 * c, o);
   }
 }
 
@@ -500,131 +602,101 @@ __global__ void __launch_bounds__(kThreads, 1)
         EBH_TRACE(kEvSReady, j);
         phase ^= 1;
         tc_fence_after();
+        // Scores in two halves of BN/2 keys: the second half's load overlaps
+        // the first half's exponentials.
+        constexpr int kHalf = BN / 16;  // column groups of 8 per half
         uint32_t sr[BN / 2];
-        if constexpr (BN == 128) {
-          tmem_ld_16x256b_x16(tS, sr);
-        } else {
-          tmem_ld_16x256b_x8(tS, sr);
-        }
+        tmem_ld_half<BN>(tS, sr);
         tmem_wait_ld();
-        if constexpr (BN == 128) {
-          reg_fence64(sr);
-        } else {
-          reg_fence32(sr);
-        }
+        reg_fence_half<BN>(sr);
+        tmem_ld_half<BN>(tS + BN / 2, sr + BN / 4);
         float* s = reinterpret_cast<float*>(sr);
-#ifdef EBH_PIPELINE_TRACE
-        {  // profiling builds: stamp only once the loaded scores are really in registers
-          const uint32_t probe = __shfl_sync(0xffffffffu, sr[BN / 2 - 1] ^ sr[0], 0);
-          EBH_TRACE(kEvSLoaded, j + (probe == 0x7fc00001u ? 1 : 0));
-        }
-#endif
+        EBH_TRACE(kEvSLoaded, j);
 
         const bool full = j >= full_lo && j < full_hi;
+        int a_lo = 0, a_hi = BN, b_lo = 0, b_hi = BN;
         if (!full) {
-          int a_lo, a_hi, b_lo, b_hi;
           row_allowed_cols(p.L, row_a, j, p.mask_kind, p.window, BN, a_lo, a_hi);
           row_allowed_cols(p.L, row_b, j, p.mask_kind, p.window, BN, b_lo, b_hi);
-#pragma unroll
-          for (int m = 0; m < BN / 8; ++m) {
-            const int c = 8 * m + 2 * t0;
-            if (c < a_lo || c >= a_hi) s[4 * m] = -INFINITY;
-            if (c + 1 < a_lo || c + 1 >= a_hi) s[4 * m + 1] = -INFINITY;
-            if (c < b_lo || c >= b_hi) s[4 * m + 2] = -INFINITY;
-            if (c + 1 < b_lo || c + 1 >= b_hi) s[4 * m + 3] = -INFINITY;
-          }
+          mask_groups<0, kHalf>(s, t0, a_lo, a_hi, b_lo, b_hi);
         }
         EBH_TRACE(kEvMasked, j);
-        // row maxima: this thread's 2 x (BN / 4) scores, then across the four
-        // threads of each row
-        float xa0 = s[0], xa1 = s[1], xb0 = s[2], xb1 = s[3];
-#pragma unroll
-        for (int m = 1; m < BN / 8; m += 2) {
-          if (m + 1 < BN / 8) {
-            xa0 = max3(xa0, s[4 * m], s[4 * m + 4]);
-            xa1 = max3(xa1, s[4 * m + 1], s[4 * m + 5]);
-            xb0 = max3(xb0, s[4 * m + 2], s[4 * m + 6]);
-            xb1 = max3(xb1, s[4 * m + 3], s[4 * m + 7]);
-          } else {
-            xa0 = fmaxf(xa0, s[4 * m]);
-            xa1 = fmaxf(xa1, s[4 * m + 1]);
-            xb0 = fmaxf(xb0, s[4 * m + 2]);
-            xb1 = fmaxf(xb1, s[4 * m + 3]);
-          }
-        }
-        float mta = fmaxf(xa0, xa1), mtb = fmaxf(xb0, xb1);
-        mta = fmaxf(mta, __shfl_xor_sync(0xffffffffu, mta, 1));
-        mtb = fmaxf(mtb, __shfl_xor_sync(0xffffffffu, mtb, 1));
-        mta = fmaxf(mta, __shfl_xor_sync(0xffffffffu, mta, 2));
-        mtb = fmaxf(mtb, __shfl_xor_sync(0xffffffffu, mtb, 2));
-        mta *= cl2;
-        mtb *= cl2;
-        // lazy rescale, per row (the four threads of a row decide alike)
-        float alpha_a = 1.f, alpha_b = 1.f;
-        bool rescale = false;
-        if (m_a == -INFINITY) {
-          m_a = mta;  // nothing accumulated for this row yet
-        } else if (mta > m_a + kRescaleThreshold) {
-          alpha_a = ex2_approx(m_a - mta);
-          m_a = mta;
-          rescale = true;
-        }
-        if (m_b == -INFINITY) {
-          m_b = mtb;
-        } else if (mtb > m_b + kRescaleThreshold) {
-          alpha_b = ex2_approx(m_b - mtb);
-          m_b = mtb;
-          rescale = true;
-        }
-        if (__any_sync(0xffffffffu, rescale)) {
-          l_a *= alpha_a; lr_a *= alpha_a;
-          l_b *= alpha_b; lr_b *= alpha_b;
-          // O_t's previous product is complete (it was issued before S_t(j))
-#pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[16];
-            tmem_ld_16x256b_x4(tO + 32 * c, o);
-            tmem_wait_ld();
-            reg_fence16(o);
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              o[i] = __float_as_uint(__uint_as_float(o[i]) * ((i & 2) ? alpha_b : alpha_a));
-            tmem_st_16x256b_x4(tO + 32 * c, o);
-          }
-        }
-        const float sa = m_a == -INFINITY ? 0.f : m_a;
-        const float sb = m_b == -INFINITY ? 0.f : m_b;
-        EBH_TRACE(kEvMaxDone, j);
-        // probabilities -> packed bf16 over the first half of S_t, four
-        // column groups (16 packed columns) per store
-#pragma unroll
-        for (int ch = 0; ch < BN / 32; ++ch) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int mm = 0; mm < 4; ++mm) {
-            const int m = 4 * ch + mm;
-            float x0, x1, x2, x3, p0, p1, p2, p3;
-            fma2(x0, x1, s[4 * m], s[4 * m + 1], cl2, cl2, -sa, -sa);
-            fma2(x2, x3, s[4 * m + 2], s[4 * m + 3], cl2, cl2, -sb, -sb);
-            if (kPolyEvery > 0 && full && (m % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
-              // this group's exponentials on the FMA pipe (no -inf here: the
-              // tile has no masked element)
-              exp2_poly2(x0, x1, p0, p1);
-              exp2_poly2(x2, x3, p2, p3);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-              p2 = ex2_approx(x2);
-              p3 = ex2_approx(x3);
+
+        // The branch must be warp-uniform: both sides run warp-collective
+        // tensor-memory instructions and shuffles.
+        if (__all_sync(0xffffffffu, m_a != -INFINITY && m_b != -INFINITY)) {
+          // Speculate that the stale reference max still holds (the tile max
+          // exceeds it by at most the threshold): the exponentials need not
+          // wait for this tile's row max.
+          const float l_a0 = l_a, l_b0 = l_b, lr_a0 = lr_a, lr_b0 = lr_b;
+          EBH_TRACE(kEvMaxDone, j);
+          probabilities<0, kHalf>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
+          tmem_wait_ld();
+          reg_fence_half<BN>(sr + BN / 4);
+          if (!full) mask_groups<kHalf, 2 * kHalf>(s, t0, a_lo, a_hi, b_lo, b_hi);
+          probabilities<kHalf, 2 * kHalf>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
+          float mta, mtb;
+          row_max_pair<BN>(s, mta, mtb);
+          mta *= cl2;
+          mtb *= cl2;
+          const bool grow_a = mta > m_a + kRescaleThreshold;
+          const bool grow_b = mtb > m_b + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, grow_a || grow_b)) {
+            // rare: redo the tile against the grown maximum
+            float alpha_a = 1.f, alpha_b = 1.f;
+            if (grow_a) {
+              alpha_a = ex2_approx(m_a - mta);
+              m_a = mta;
             }
-            pk[2 * mm] = pack_bf16x2(p0, p1);
-            pk[2 * mm + 1] = pack_bf16x2(p2, p3);
-            add2(l_a, l_b, l_a, l_b, p0, p2);
-            add2(l_a, l_b, l_a, l_b, p1, p3);
-            acc_bf16x2_sum(lr_a, pk[2 * mm]);
-            acc_bf16x2_sum(lr_b, pk[2 * mm + 1]);
+            if (grow_b) {
+              alpha_b = ex2_approx(m_b - mtb);
+              m_b = mtb;
+            }
+            l_a = l_a0 * alpha_a;
+            lr_a = lr_a0 * alpha_a;
+            l_b = l_b0 * alpha_b;
+            lr_b = lr_b0 * alpha_b;
+            rescale_o_rows<D>(tO, alpha_a, alpha_b);
+            probabilities<0, 2 * kHalf>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
           }
-          tmem_st_16x128b_x4(tS + 16 * ch, pk);
+        } else {
+          // first key block with an allowed key for some row of this thread:
+          // take the tile max as the reference before any exponential
+          tmem_wait_ld();
+          reg_fence_half<BN>(sr + BN / 4);
+          if (!full) mask_groups<kHalf, 2 * kHalf>(s, t0, a_lo, a_hi, b_lo, b_hi);
+          float mta, mtb;
+          row_max_pair<BN>(s, mta, mtb);
+          mta *= cl2;
+          mtb *= cl2;
+          float alpha_a = 1.f, alpha_b = 1.f;
+          bool grow = false;
+          if (m_a == -INFINITY) {
+            m_a = mta;  // nothing accumulated for this row yet
+          } else if (mta > m_a + kRescaleThreshold) {
+            alpha_a = ex2_approx(m_a - mta);
+            m_a = mta;
+            grow = true;
+          }
+          if (m_b == -INFINITY) {
+            m_b = mtb;
+          } else if (mtb > m_b + kRescaleThreshold) {
+            alpha_b = ex2_approx(m_b - mtb);
+            m_b = mtb;
+            grow = true;
+          }
+          if (__any_sync(0xffffffffu, grow)) {
+            l_a *= alpha_a;
+            lr_a *= alpha_a;
+            l_b *= alpha_b;
+            lr_b *= alpha_b;
+            rescale_o_rows<D>(tO, alpha_a, alpha_b);
+          }
+          EBH_TRACE(kEvMaxDone, j);
+          // a row with every key masked so far keeps m = -inf: subtract 0 so
+          // that -inf - (-inf) never happens (its probabilities are all 0)
+          probabilities<0, 2 * kHalf>(s, cl2, m_a == -INFINITY ? 0.f : m_a,
+                                      m_b == -INFINITY ? 0.f : m_b, tS, l_a, l_b, lr_a, lr_b);
         }
         tmem_wait_st();
         tc_fence_before();
