@@ -34,7 +34,8 @@ ATTN_DTYPE_F32 = 1
 # Every entry point declared in include/attn.h.
 EXPORTED = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ex", "attn_strerror", "attn_last_cuda_error",
             "attn_device_status", "attn_selftest_wait_timeout", "attn_kv_tile_range",
-            "attn_kv_tile_class", "attn_kv_full_range", "attn_abi_version")
+            "attn_kv_tile_class", "attn_kv_full_range", "attn_splitkv_workspace_bytes",
+            "attn_fwd_splitkv", "attn_merge", "attn_abi_version")
 
 
 class AttnParams(ctypes.Structure):
@@ -96,9 +97,14 @@ def _load():
             lib.attn_kv_full_range.argtypes = [i, i, i, i, i, i, ctypes.POINTER(i),
                                                ctypes.POINTER(i)]
             lib.attn_abi_version.argtypes = []
+            lib.attn_splitkv_workspace_bytes.argtypes = [i, i, i, i, i]
+            lib.attn_fwd_splitkv.argtypes = [ctypes.POINTER(AttnParams), i, vp, ctypes.c_size_t, vp]
+            lib.attn_merge.argtypes = [vp, vp, i, ctypes.POINTER(i), i, i, vp, vp, i, i, i, i, i,
+                                       vp]
             for name in EXPORTED:
                 if name != "attn_strerror":
                     getattr(lib, name).restype = ctypes.c_int
+            lib.attn_splitkv_workspace_bytes.restype = ctypes.c_size_t
             _lib = lib
     return _lib
 
@@ -162,6 +168,94 @@ def forward(q, k, v, scale=None, mask="none", window=0, block_n=0, out=None, lse
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_ex")
     return out, (lse if want_lse else None)
+
+
+def _params(q, k, v, scale, mask, window, block_n, out, lse, want_lse, wait_timeout_ns):
+    import torch
+
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("q, k, v must be bf16 or fp32")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share one [B, H, L, d] shape")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    B, H, L, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if mask not in MASK_KINDS:
+        raise ValueError(f"mask must be one of {sorted(MASK_KINDS)}")
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    p = AttnParams()
+    p.dtype = ATTN_DTYPE_BF16 if q.dtype == torch.bfloat16 else ATTN_DTYPE_F32
+    p.q, p.k, p.v, p.out = q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr()
+    p.lse = lse.data_ptr() if (want_lse and lse is not None) else None
+    p.B, p.H, p.L, p.d = B, H, L, d
+    p.scale = float(scale)
+    p.mask_kind = MASK_KINDS[mask]
+    p.window = int(window)
+    p.block_n = int(block_n)
+    p.wait_timeout_ns = int(wait_timeout_ns)
+    return p, out, lse
+
+
+def splitkv_workspace_bytes(B, H, L, d, num_splits) -> int:
+    """Bytes of workspace attn_fwd_splitkv needs for num_splits key runs."""
+    return int(_load().attn_splitkv_workspace_bytes(B, H, L, d, num_splits))
+
+
+def forward_splitkv(q, k, v, num_splits, scale=None, mask="none", window=0, block_n=0,
+                    out=None, lse=None, want_lse=True, workspace=None, stream=None):
+    """forward() with the key blocks cut into up to num_splits runs that run as
+    separate work units, then merged exactly.  bf16 only.  `workspace` is a
+    CUDA uint8 tensor of at least splitkv_workspace_bytes(...) bytes (allocated
+    here when omitted)."""
+    import torch
+
+    p, out, lse = _params(q, k, v, scale, mask, window, block_n, out, lse, want_lse, 0)
+    B, H, L, d = q.shape
+    need = splitkv_workspace_bytes(B, H, L, d, num_splits)
+    if workspace is None:
+        workspace = torch.empty(need + 256, dtype=torch.uint8, device=q.device)
+    base = workspace.data_ptr()
+    pad = (-base) % 256
+    with torch.cuda.device(q.device):
+        st = _load().attn_fwd_splitkv(ctypes.byref(p), int(num_splits),
+                                      ctypes.c_void_p(base + pad), workspace.numel() - pad,
+                                      _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_splitkv")
+    return out, (lse if want_lse else None)
+
+
+def merge(o_parts, lse_parts, split_bounds, mask="none", window=0, out_dtype=None, out=None,
+          lse=None, stream=None):
+    """Exact merge of partials over disjoint key ranges (see attn_merge in
+    include/attn.h).  o_parts: fp32 [S,B,H,L,d] CUDA; lse_parts: fp32 [S,B,H,L];
+    split_bounds: S+1 ints from 0 to L."""
+    import torch
+
+    S, B, H, L, d = o_parts.shape
+    if out_dtype is None:
+        out_dtype = torch.bfloat16
+    if out is None:
+        out = torch.empty((B, H, L, d), dtype=out_dtype, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=o_parts.device)
+    bounds = (ctypes.c_int * (S + 1))(*[int(b) for b in split_bounds])
+    dt = ATTN_DTYPE_BF16 if out.dtype == torch.bfloat16 else ATTN_DTYPE_F32
+    with torch.cuda.device(o_parts.device):
+        st = _load().attn_merge(o_parts.data_ptr(), lse_parts.data_ptr(), S, bounds,
+                                MASK_KINDS[mask], int(window), out.data_ptr(), lse.data_ptr(),
+                                dt, B, H, L, d, _stream_handle(stream, o_parts.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_merge")
+    return out, lse
 
 
 def device_status(device: int = 0, reset: bool = True) -> int:

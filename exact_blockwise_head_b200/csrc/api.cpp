@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstddef>
 #include <cstdint>
 #include <mutex>
 
@@ -213,6 +214,111 @@ int attn_kv_tile_class(int L, int q_first, int q_last, int j, int mask_kind, int
   if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_WINDOW) return -ATTN_ERR_INVALID;
   if (mask_kind == ATTN_MASK_WINDOW && window < 0) return -ATTN_ERR_INVALID;
   return ebh::kv_tile_class(L, q_first, q_last, j, mask_kind, window, block_n);
+}
+
+size_t attn_splitkv_workspace_bytes(int B, int H, int L, int d, int num_splits) {
+  if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || num_splits < 1) return 0;
+  const size_t rows = static_cast<size_t>(num_splits) * B * H * L;
+  const size_t o_bytes = (rows * d * sizeof(float) + 255) / 256 * 256;
+  return o_bytes + rows * sizeof(float);
+}
+
+int attn_fwd_splitkv(const attn_params* p, int num_splits, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  ebh::FwdArgs a;
+  int st = validate(p, &a);
+  if (st != ATTN_OK) return st;
+  if (p->dtype != ATTN_DTYPE_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (num_splits < 1 || num_splits > ebh::kMaxSplits) return ATTN_ERR_INVALID;
+  // whole key blocks per split; the last split may be shorter
+  const int nkv = (a.L + a.block_n - 1) / a.block_n;
+  const int split_blocks = (nkv + num_splits - 1) / num_splits;
+  const int splits = (nkv + split_blocks - 1) / split_blocks;
+  if (splits == 1) return attn_fwd_ex(p, stream);
+  const size_t need = attn_splitkv_workspace_bytes(a.B, a.H, a.L, a.d, splits);
+  if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_INVALID;
+  if (!aligned(workspace, 256)) return ATTN_ERR_MISALIGNED;
+  const size_t rows = static_cast<size_t>(splits) * a.B * a.H * a.L;
+  const size_t o_bytes = (rows * a.d * sizeof(float) + 255) / 256 * 256;
+  float* o_part = static_cast<float*>(workspace);
+  float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + o_bytes);
+  {  // the workspace must not alias the problem's tensors
+    const uint64_t tb = static_cast<uint64_t>(a.B) * a.H * a.L * a.d * 2;
+    const uint64_t lb = static_cast<uint64_t>(a.B) * a.H * a.L * 4;
+    if (overlap(workspace, need, p->q, tb) || overlap(workspace, need, p->k, tb) ||
+        overlap(workspace, need, p->v, tb) || overlap(workspace, need, p->out, tb) ||
+        (p->lse && overlap(workspace, need, p->lse, lb)))
+      return ATTN_ERR_INVALID;
+  }
+  if ((st = check_device_sm100()) != ATTN_OK) return st;
+  a.num_splits = splits;
+  a.split_keys = split_blocks * a.block_n;
+  a.o_part = o_part;
+  a.lse_part = lse_part;
+  cudaError_t err = cudaSuccess;
+  st = ebh::launch_fwd_bf16_sm100(a, static_cast<cudaStream_t>(stream), &err);
+  if (st != ATTN_OK) {
+    if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
+    return st;
+  }
+  ebh::MergeArgs m = {};
+  m.o_part = o_part;
+  m.lse_part = lse_part;
+  m.num_splits = splits;
+  for (int s = 0; s <= splits; ++s) {
+    const long long b = static_cast<long long>(s) * a.split_keys;
+    m.bounds[s] = static_cast<int>(b < a.L ? b : a.L);
+  }
+  m.out = a.out;
+  m.lse = a.lse;
+  m.out_f32 = false;
+  m.BH = a.B * a.H;
+  m.L = a.L;
+  m.d = a.d;
+  m.mask_kind = a.mask_kind;
+  m.window = a.window;
+  st = ebh::launch_merge(m, static_cast<cudaStream_t>(stream), &err);
+  if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
+  return st;
+}
+
+int attn_merge(const float* o_parts, const float* lse_parts, int num_splits,
+               const int* split_bounds, int mask_kind, int window, void* out, float* lse,
+               int out_dtype, int B, int H, int L, int d, void* stream) {
+  if (!o_parts || !lse_parts || !split_bounds || !out) return ATTN_ERR_INVALID;
+  if (num_splits < 1 || num_splits > ebh::kMaxSplits) return ATTN_ERR_INVALID;
+  if (B <= 0 || H <= 0 || L <= 0) return ATTN_ERR_INVALID;
+  if (static_cast<long long>(B) * H > 0x7fffffffLL) return ATTN_ERR_INVALID;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_WINDOW) return ATTN_ERR_INVALID;
+  if (mask_kind == ATTN_MASK_WINDOW && window < 0) return ATTN_ERR_INVALID;
+  if (out_dtype != ATTN_DTYPE_BF16 && out_dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (split_bounds[0] != 0) return ATTN_ERR_INVALID;
+  for (int s = 0; s < num_splits; ++s)
+    if (split_bounds[s + 1] < split_bounds[s]) return ATTN_ERR_INVALID;
+  if (split_bounds[num_splits] != L) return ATTN_ERR_INVALID;
+  if (!aligned(o_parts, 16) || !aligned(lse_parts, 4) || !aligned(out, 16) ||
+      (lse && !aligned(lse, 4)))
+    return ATTN_ERR_MISALIGNED;
+  int st = check_device_sm100();
+  if (st != ATTN_OK) return st;
+  ebh::MergeArgs m = {};
+  m.o_part = o_parts;
+  m.lse_part = lse_parts;
+  m.num_splits = num_splits;
+  for (int s = 0; s <= num_splits; ++s) m.bounds[s] = split_bounds[s];
+  m.out = out;
+  m.lse = lse;
+  m.out_f32 = out_dtype == ATTN_DTYPE_F32;
+  m.BH = B * H;
+  m.L = L;
+  m.d = d;
+  m.mask_kind = mask_kind;
+  m.window = mask_kind == ATTN_MASK_WINDOW ? (window > L ? L : window) : 0;
+  cudaError_t err = cudaSuccess;
+  st = ebh::launch_merge(m, static_cast<cudaStream_t>(stream), &err);
+  if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
+  return st;
 }
 
 int attn_kv_full_range(int L, int q_first, int q_last, int mask_kind, int window, int block_n,

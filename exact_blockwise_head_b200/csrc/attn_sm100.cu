@@ -58,6 +58,19 @@ constexpr int kSoftmaxRegs = 104;
 constexpr int kOtherRegs = 64;
 static_assert(kSoftmaxRegs * kNQ * kSoftmaxThreads + kOtherRegs * 128 <= kLaunchRegs * kThreads,
               "register split exceeds the launch allocation");
+// Tuning knobs of the softmax arithmetic.  kPolyEvery: one column group of
+// eight in kPolyEvery takes its exponentials from a polynomial on the FMA pipe
+// instead of the MUFU pipe (tiles without masked elements only; 0 = none).
+// kScalarMath: scalar fp32 FMA/add instead of the paired f32x2 forms.
+#ifndef EBH_POLY_EVERY
+#define EBH_POLY_EVERY 0
+#endif
+#ifndef EBH_SCALAR_MATH
+#define EBH_SCALAR_MATH 0
+#endif
+constexpr int kPolyEvery = EBH_POLY_EVERY > 0 ? EBH_POLY_EVERY : 1;
+constexpr bool kPolyOn = EBH_POLY_EVERY > 0;
+constexpr bool kScalarMath = EBH_SCALAR_MATH != 0;
 // Lazy rescale: keep the stale max until the row max exceeds it by more than
 // 2^8 (probabilities then stay <= 256, far inside fp32/bf16 range).
 constexpr float kRescaleThreshold = 8.0f;
@@ -129,48 +142,19 @@ struct Params {
   float scale_log2;  // scale * log2(e)
   int num_units, nqp;
   uint64_t timeout_ns;
+  // Split-KV mode (o_part != nullptr): the key blocks are cut into runs of
+  // split_blocks; unit u covers split u % num_splits, and writes its fp32
+  // partial O (normalised within the split) and partial LSE to
+  // o_part[s][bh][row][:] and lse_part[s][bh][row] instead of out / lse.
+  int num_splits, split_blocks;
+  float* o_part;
+  float* lse_part;
 };
 
-struct Unit {
-  int bh, qp;
-  bool valid[kNQ];
-  int q_first[kNQ], q_last[kNQ], lo[kNQ], hi[kNQ];
-  int ulo, uhi;  // union of the two key-block ranges
-};
-
-template <int BN>
-__device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
-  Unit w;
-  if (p.mask_kind == kMaskCausal) {
-    // longest units first: causal work grows with the query position
-    w.qp = p.nqp - 1 - u / p.BH;
-    w.bh = u % p.BH;
-  } else {
-    w.bh = u / p.nqp;
-    w.qp = u % p.nqp;
-  }
-  w.ulo = 0x7fffffff;
-  w.uhi = 0;
-#pragma unroll
-  for (int t = 0; t < kNQ; ++t) {
-    w.q_first[t] = w.qp * kUnitRows + t * kBM;
-    w.valid[t] = w.q_first[t] < p.L;
-    w.q_last[t] = min(w.q_first[t] + kBM - 1, p.L - 1);
-    w.lo[t] = w.hi[t] = 0;
-    if (w.valid[t]) {
-      kv_tile_range(p.L, w.q_first[t], w.q_last[t], p.mask_kind, p.window, BN, w.lo[t], w.hi[t]);
-      w.ulo = min(w.ulo, w.lo[t]);
-      w.uhi = max(w.uhi, w.hi[t]);
-    }
-  }
-  if (w.uhi <= w.ulo) w.ulo = w.uhi = 0;
-  return w;
-}
-
-// One Q tile of unit u, decoded on its own (no per-tile arrays, so the
-// softmax threads, whose tile index is a run-time value, keep it in registers).
+// One Q tile of unit u: its head, first/last query row and the key blocks
+// [lo, hi) it must visit (empty -> the tile does no work in this unit).
 struct TileWork {
-  int bh;
+  int bh, split;
   bool valid;
   int q_first, q_last, lo, hi;
 };
@@ -178,8 +162,14 @@ struct TileWork {
 template <int BN>
 __device__ __forceinline__ TileWork decode_tile(int u, int t, const Params& p) {
   TileWork w;
+  w.split = 0;
+  if (p.num_splits > 1) {
+    w.split = u % p.num_splits;
+    u /= p.num_splits;
+  }
   int qp;
   if (p.mask_kind == kMaskCausal) {
+    // longest units first: causal work grows with the query position
     qp = p.nqp - 1 - u / p.BH;
     w.bh = u % p.BH;
   } else {
@@ -190,7 +180,46 @@ __device__ __forceinline__ TileWork decode_tile(int u, int t, const Params& p) {
   w.valid = w.q_first < p.L;
   w.q_last = min(w.q_first + kBM - 1, p.L - 1);
   w.lo = w.hi = 0;
-  if (w.valid) kv_tile_range(p.L, w.q_first, w.q_last, p.mask_kind, p.window, BN, w.lo, w.hi);
+  if (w.valid) {
+    kv_tile_range(p.L, w.q_first, w.q_last, p.mask_kind, p.window, BN, w.lo, w.hi);
+    if (p.num_splits > 1) {
+      w.lo = max(w.lo, w.split * p.split_blocks);
+      w.hi = min(w.hi, (w.split + 1) * p.split_blocks);
+      if (w.hi <= w.lo) {
+        w.valid = false;
+        w.lo = w.hi = 0;
+      }
+    }
+  }
+  return w;
+}
+
+struct Unit {
+  int bh;
+  bool valid[kNQ];
+  int q_first[kNQ], lo[kNQ], hi[kNQ];
+  int ulo, uhi;  // union of the two key-block ranges
+};
+
+template <int BN>
+__device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
+  Unit w;
+  w.ulo = 0x7fffffff;
+  w.uhi = 0;
+#pragma unroll
+  for (int t = 0; t < kNQ; ++t) {
+    const TileWork tw = decode_tile<BN>(u, t, p);
+    w.bh = tw.bh;
+    w.valid[t] = tw.valid;
+    w.q_first[t] = tw.q_first;
+    w.lo[t] = tw.lo;
+    w.hi[t] = tw.hi;
+    if (tw.valid) {
+      w.ulo = min(w.ulo, tw.lo);
+      w.uhi = max(w.uhi, tw.hi);
+    }
+  }
+  if (w.uhi <= w.ulo) w.ulo = w.uhi = 0;
   return w;
 }
 
@@ -280,7 +309,7 @@ __device__ __forceinline__ void row_max_pair(const float* s, float& mta, float& 
 // p = 2^(s cl2 - m) for column groups [G0, G1) (multiples of 4), packed to bf16
 // and written over the first half of S_t (group m -> packed column 4m + t0);
 // l += p, lr += bf16(p), per row.
-template <int G0, int G1>
+template <int G0, int G1, bool kPoly>
 __device__ __forceinline__ void probabilities(const float* s, float cl2, float ma, float mb,
                                               uint32_t tS, float& l_a, float& l_b, float& lr_a,
                                               float& lr_b) {
@@ -290,15 +319,36 @@ __device__ __forceinline__ void probabilities(const float* s, float cl2, float m
 #pragma unroll
     for (int mm = 0; mm < 4; ++mm) {
       const int m = 4 * ch + mm;
-      float x0, x1, x2, x3;
-      fma2(x0, x1, s[4 * m], s[4 * m + 1], cl2, cl2, -ma, -ma);
-      fma2(x2, x3, s[4 * m + 2], s[4 * m + 3], cl2, cl2, -mb, -mb);
-      const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-      const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+      float x0, x1, x2, x3, p0, p1, p2, p3;
+      if constexpr (kScalarMath) {
+        x0 = fmaf(s[4 * m], cl2, -ma);
+        x1 = fmaf(s[4 * m + 1], cl2, -ma);
+        x2 = fmaf(s[4 * m + 2], cl2, -mb);
+        x3 = fmaf(s[4 * m + 3], cl2, -mb);
+      } else {
+        fma2(x0, x1, s[4 * m], s[4 * m + 1], cl2, cl2, -ma, -ma);
+        fma2(x2, x3, s[4 * m + 2], s[4 * m + 3], cl2, cl2, -mb, -mb);
+      }
+      if (kPoly && (m % kPolyEvery) == kPolyEvery - 1) {
+        exp2_poly2(x0, x1, p0, p1);
+        exp2_poly2(x2, x3, p2, p3);
+      } else {
+        p0 = ex2_approx(x0);
+        p1 = ex2_approx(x1);
+        p2 = ex2_approx(x2);
+        p3 = ex2_approx(x3);
+      }
       pk[2 * mm] = pack_bf16x2(p0, p1);
       pk[2 * mm + 1] = pack_bf16x2(p2, p3);
-      add2(l_a, l_b, l_a, l_b, p0, p2);
-      add2(l_a, l_b, l_a, l_b, p1, p3);
+      if constexpr (kScalarMath) {
+        l_a += p0;
+        l_b += p2;
+        l_a += p1;
+        l_b += p3;
+      } else {
+        add2(l_a, l_b, l_a, l_b, p0, p2);
+        add2(l_a, l_b, l_a, l_b, p1, p3);
+      }
       acc_bf16x2_sum(lr_a, pk[2 * mm]);
       acc_bf16x2_sum(lr_b, pk[2 * mm + 1]);
     }
@@ -494,9 +544,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             lo0 = w0.lo; hi0 = w0.valid ? w0.hi : w0.lo;
             lo1 = w1.lo; hi1 = w1.valid ? w1.hi : w1.lo;
           }
-          const bool has1 = hi1 > lo1;
-          const int ulo = has1 ? min(lo0, lo1) : lo0;
-          const int uhi = has1 ? max(hi0, hi1) : hi0;
+          const bool has0 = hi0 > lo0, has1 = hi1 > lo1;
+          const int ulo = has0 ? (has1 ? min(lo0, lo1) : lo0) : (has1 ? lo1 : 0);
+          const int uhi = has0 ? (has1 ? max(hi0, hi1) : hi0) : (has1 ? hi1 : 0);
           int pend_v = -1;  // ring stage of V_(j-1) still owed a P_1 . V product
           for (int j = ulo; ok && j < uhi; ++j) {
             const int kst = kv_it % C::kStages;
@@ -555,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           // Q tiles and O accumulators used by this unit move to their next phase
-          const uint32_t used = (hi0 > lo0 ? 1u : 0u) | (has1 ? 2u : 0u);
+          const uint32_t used = (has0 ? 1u : 0u) | (has1 ? 2u : 0u);
           par_q ^= used;
           par_oe ^= used;
         }
@@ -630,11 +680,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           // wait for this tile's row max.
           const float l_a0 = l_a, l_b0 = l_b, lr_a0 = lr_a, lr_b0 = lr_b;
           EBH_TRACE(kEvMaxDone, j);
-          probabilities<0, kHalf>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
+          if (full) {
+            probabilities<0, kHalf, kPolyOn>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
+          } else {
+            probabilities<0, kHalf, false>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
+          }
           tmem_wait_ld();
           reg_fence_half<BN>(sr + BN / 4);
           if (!full) mask_groups<kHalf, 2 * kHalf>(s, t0, a_lo, a_hi, b_lo, b_hi);
-          probabilities<kHalf, 2 * kHalf>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
+          if (full) {
+            probabilities<kHalf, 2 * kHalf, kPolyOn>(s, cl2, m_a, m_b, tS, l_a, l_b,
+                                                               lr_a, lr_b);
+          } else {
+            probabilities<kHalf, 2 * kHalf, false>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
+          }
           float mta, mtb;
           row_max_pair<BN>(s, mta, mtb);
           mta *= cl2;
@@ -657,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             l_b = l_b0 * alpha_b;
             lr_b = lr_b0 * alpha_b;
             rescale_o_rows<D>(tO, alpha_a, alpha_b);
-            probabilities<0, 2 * kHalf>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
+            probabilities<0, 2 * kHalf, false>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
           }
         } else {
           // first key block with an allowed key for some row of this thread:
@@ -695,7 +754,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           EBH_TRACE(kEvMaxDone, j);
           // a row with every key masked so far keeps m = -inf: subtract 0 so
           // that -inf - (-inf) never happens (its probabilities are all 0)
-          probabilities<0, 2 * kHalf>(s, cl2, m_a == -INFINITY ? 0.f : m_a,
+          probabilities<0, 2 * kHalf, false>(s, cl2, m_a == -INFINITY ? 0.f : m_a,
                                       m_b == -INFINITY ? 0.f : m_b, tS, l_a, l_b, lr_a, lr_b);
         }
         tmem_wait_st();
@@ -722,36 +781,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_a = lr_a > 0.f ? 1.f / lr_a : 0.f;
       const float inv_b = lr_b > 0.f ? 1.f / lr_b : 0.f;
       const bool ok_a = row_a < p.L, ok_b = row_b < p.L;
-      uint32_t* dst_a = reinterpret_cast<uint32_t*>(
-          static_cast<uint16_t*>(p.out) +
-          (static_cast<size_t>(w.bh) * p.L + (ok_a ? row_a : 0)) * D);
-      uint32_t* dst_b = reinterpret_cast<uint32_t*>(
-          static_cast<uint16_t*>(p.out) +
-          (static_cast<size_t>(w.bh) * p.L + (ok_b ? row_b : 0)) * D);
+      const float lse_a = l_a > 0.f ? (m_a + log2f(l_a)) * 0.69314718055994531f : -INFINITY;
+      const float lse_b = l_b > 0.f ? (m_b + log2f(l_b)) * 0.69314718055994531f : -INFINITY;
+      if (p.o_part == nullptr) {
+        uint32_t* dst_a = reinterpret_cast<uint32_t*>(
+            static_cast<uint16_t*>(p.out) +
+            (static_cast<size_t>(w.bh) * p.L + (ok_a ? row_a : 0)) * D);
+        uint32_t* dst_b = reinterpret_cast<uint32_t*>(
+            static_cast<uint16_t*>(p.out) +
+            (static_cast<size_t>(w.bh) * p.L + (ok_b ? row_b : 0)) * D);
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[16];
-        tmem_ld_16x256b_x4(tO + 32 * c, o);
-        tmem_wait_ld();
-        reg_fence16(o);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[16];
+          tmem_ld_16x256b_x4(tO + 32 * c, o);
+          tmem_wait_ld();
+          reg_fence16(o);
 #pragma unroll
-        for (int mm = 0; mm < 4; ++mm) {
-          const int col2 = (32 * c + 8 * mm + 2 * t0) / 2;  // pair index in the row
-          const uint32_t va = pack_bf16x2(__uint_as_float(o[4 * mm]) * inv_a,
-                                          __uint_as_float(o[4 * mm + 1]) * inv_a);
-          const uint32_t vb = pack_bf16x2(__uint_as_float(o[4 * mm + 2]) * inv_b,
-                                          __uint_as_float(o[4 * mm + 3]) * inv_b);
-          if (ok_a) dst_a[col2] = va;
-          if (ok_b) dst_b[col2] = vb;
+          for (int mm = 0; mm < 4; ++mm) {
+            const int col2 = (32 * c + 8 * mm + 2 * t0) / 2;  // pair index in the row
+            const uint32_t va = pack_bf16x2(__uint_as_float(o[4 * mm]) * inv_a,
+                                            __uint_as_float(o[4 * mm + 1]) * inv_a);
+            const uint32_t vb = pack_bf16x2(__uint_as_float(o[4 * mm + 2]) * inv_b,
+                                            __uint_as_float(o[4 * mm + 3]) * inv_b);
+            if (ok_a) dst_a[col2] = va;
+            if (ok_b) dst_b[col2] = vb;
+          }
         }
-      }
-      if (t0 == 0 && p.lse != nullptr) {
-        if (ok_a)
-          p.lse[static_cast<size_t>(w.bh) * p.L + row_a] =
-              l_a > 0.f ? (m_a + log2f(l_a)) * 0.69314718055994531f : -INFINITY;
-        if (ok_b)
-          p.lse[static_cast<size_t>(w.bh) * p.L + row_b] =
-              l_b > 0.f ? (m_b + log2f(l_b)) * 0.69314718055994531f : -INFINITY;
+        if (t0 == 0 && p.lse != nullptr) {
+          if (ok_a) p.lse[static_cast<size_t>(w.bh) * p.L + row_a] = lse_a;
+          if (ok_b) p.lse[static_cast<size_t>(w.bh) * p.L + row_b] = lse_b;
+        }
+      } else {
+        // split-KV partial: fp32 O normalised within the split, and its LSE
+        const size_t head = static_cast<size_t>(w.split) * p.BH + w.bh;
+        float2* dst_a = reinterpret_cast<float2*>(
+            p.o_part + (head * p.L + (ok_a ? row_a : 0)) * D);
+        float2* dst_b = reinterpret_cast<float2*>(
+            p.o_part + (head * p.L + (ok_b ? row_b : 0)) * D);
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[16];
+          tmem_ld_16x256b_x4(tO + 32 * c, o);
+          tmem_wait_ld();
+          reg_fence16(o);
+#pragma unroll
+          for (int mm = 0; mm < 4; ++mm) {
+            const int col2 = (32 * c + 8 * mm + 2 * t0) / 2;
+            if (ok_a)
+              dst_a[col2] = make_float2(__uint_as_float(o[4 * mm]) * inv_a,
+                                        __uint_as_float(o[4 * mm + 1]) * inv_a);
+            if (ok_b)
+              dst_b[col2] = make_float2(__uint_as_float(o[4 * mm + 2]) * inv_b,
+                                        __uint_as_float(o[4 * mm + 3]) * inv_b);
+          }
+        }
+        if (t0 == 0) {
+          if (ok_a) p.lse_part[head * p.L + row_a] = lse_a;
+          if (ok_b) p.lse_part[head * p.L + row_b] = lse_b;
+        }
       }
       tc_fence_before();
       EBH_TRACE(kEvEpilogueDone, 0);
@@ -886,7 +973,17 @@ int launch_t(const FwdArgs& a, cudaStream_t stream, cudaError_t* err) {
   p.window = a.window;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.nqp = (a.L + kUnitRows - 1) / kUnitRows;
-  const long long units = static_cast<long long>(BH) * p.nqp;
+  p.num_splits = 1;
+  p.split_blocks = 0;
+  p.o_part = nullptr;
+  p.lse_part = nullptr;
+  if (a.o_part != nullptr) {
+    p.num_splits = a.num_splits;
+    p.split_blocks = a.split_keys / BN;
+    p.o_part = a.o_part;
+    p.lse_part = a.lse_part;
+  }
+  const long long units = static_cast<long long>(BH) * p.nqp * p.num_splits;
   if (units > 0x7fffffffLL) {
     *err = cudaErrorInvalidValue;
     return ATTN_ERR_UNSUPPORTED;

@@ -20,12 +20,37 @@ struct FwdArgs {
   int window;       // already clamped to [0, L]
   int block_n;      // 64 or 128 on the bf16 path
   uint64_t timeout_ns;
+  // split-KV partial mode (bf16 path): when o_part is set, the keys are cut
+  // into num_splits runs of split_keys (a multiple of block_n) and the kernel
+  // writes fp32 partial O [S,B,H,L,d] and partial LSE [S,B,H,L] instead of
+  // out / lse.
+  int num_splits = 1;
+  int split_keys = 0;
+  float* o_part = nullptr;
+  float* lse_part = nullptr;
+};
+
+// Merge of split-KV partials: for every row, the splits whose key range
+// [bounds[s], bounds[s+1]) holds an allowed key of the row are combined,
+// O = sum_s e^(LSE_s - LSE) O_s, LSE = ln sum_s e^(LSE_s).
+constexpr int kMaxSplits = 64;
+struct MergeArgs {
+  const float* o_part;
+  const float* lse_part;
+  int num_splits;
+  int bounds[kMaxSplits + 1];
+  void* out;           // bf16 or fp32 [B,H,L,d]
+  float* lse;          // fp32 [B,H,L] or nullptr
+  bool out_f32;
+  int BH, L, d;
+  int mask_kind, window;
 };
 
 // Each returns an ATTN_* status; on ATTN_ERR_CUDA *err holds the CUDA code.
 int launch_fwd_bf16_sm100(const FwdArgs& a, cudaStream_t stream, cudaError_t* err);
 int launch_fwd_f32(const FwdArgs& a, cudaStream_t stream, cudaError_t* err);
 int launch_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream, cudaError_t* err);
+int launch_merge(const MergeArgs& m, cudaStream_t stream, cudaError_t* err);
 int read_device_status(int device, int reset, cudaError_t* err);
 
 }  // namespace ebh

@@ -44,6 +44,7 @@
 #ifndef EBH_ATTN_H
 #define EBH_ATTN_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -165,6 +166,41 @@ ATTN_API int attn_kv_tile_class(int L, int q_first, int q_last, int j, int mask_
  * the kernels test j against it instead of classifying every block. */
 ATTN_API int attn_kv_full_range(int L, int q_first, int q_last, int mask_kind, int window,
                                 int block_n, int* lo, int* hi);
+
+/*
+ * Split-KV forward (bf16 path).  The key blocks are cut into up to
+ * num_splits (1..64) contiguous runs; every (query tile, run) pair is an
+ * independent work unit, which keeps all SMs busy when B*H*L/256 is small.
+ * Each run writes an fp32 partial output normalised within the run and its
+ * LSE into `workspace`, then attn_merge's rule combines the runs exactly
+ * (the "tree reduction" of local attention results, page "Mosaic multi-GPU
+ * sequence-sharded attention", section 2.1).  The workspace is device memory
+ * owned by the caller, 256-byte aligned, at least
+ * attn_splitkv_workspace_bytes(B, H, L, d, runs) bytes (runs = the number of
+ * runs actually used, never more than num_splits; passing num_splits there is
+ * always enough); it must not overlap any other argument.  Its contents on
+ * entry do not matter.  With one run this is attn_fwd_ex and the workspace
+ * is not touched.  Other arguments and errors as attn_fwd_ex.
+ */
+ATTN_API size_t attn_splitkv_workspace_bytes(int B, int H, int L, int d, int num_splits);
+ATTN_API int attn_fwd_splitkv(const attn_params* p, int num_splits, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
+ * Exact merge of partial results over disjoint key ranges:
+ *   LSE_i = ln sum_s exp(LSE_s,i),  O_i = sum_s exp(LSE_s,i - LSE_i) O_s,i
+ * over the splits s whose key range [split_bounds[s], split_bounds[s+1])
+ * holds a key that row i may attend to under (mask_kind, window); other
+ * splits are not read for that row.  o_parts: fp32 [S,B,H,L,d] (16-byte
+ * aligned), each partial normalised within its range; lse_parts: fp32
+ * [S,B,H,L].  split_bounds: host array of S+1 increasing key indices from 0
+ * to L.  out: [B,H,L,d] in out_dtype (ATTN_DTYPE_BF16 rounds to nearest
+ * even); lse: fp32 [B,H,L] or NULL.  d in {64, 128}, 1 <= S <= 64.
+ * Asynchronous on `stream`; allocates nothing.
+ */
+ATTN_API int attn_merge(const float* o_parts, const float* lse_parts, int num_splits,
+                        const int* split_bounds, int mask_kind, int window, void* out,
+                        float* lse, int out_dtype, int B, int H, int L, int d, void* stream);
 
 /* ATTN_ABI_VERSION of the loaded library. */
 ATTN_API int attn_abi_version(void);

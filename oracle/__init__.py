@@ -56,8 +56,10 @@ def _bind(path):
     for name in ("oracle_attn_kv_blockwise", "oracle_attn_q_blockwise"):
         getattr(lib, name).argtypes = [f32p, f32p, f32p, f64p, f64p, i64, i64, i64, i64,
                                        ctypes.c_double, ctypes.c_int, i64, i64]
+    lib.oracle_attn_partial.argtypes = [f32p, f32p, f32p, f64p, f64p, i64, i64, i64, i64,
+                                        ctypes.c_double, ctypes.c_int, i64, i64, i64]
     for name in ("oracle_attn_fwd", "oracle_attn_rows", "oracle_attn_kv_blockwise",
-                 "oracle_attn_q_blockwise"):
+                 "oracle_attn_q_blockwise", "oracle_attn_partial"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -160,6 +162,20 @@ class Oracle:
         return self._blockwise("oracle_attn_q_blockwise", q, k, v, block, scale, mask, window)
 
 
+    def attention_partial(self, q, k, v, key_lo, key_hi, scale=None, mask="none", window=0):
+        """The definition over keys [key_lo, key_hi) only (single thread)."""
+        q, k, v, B, H, L, d, scale, mk, w = _common(q, k, v, scale, mask, window)
+        out = np.empty((B, H, L, d), np.float64)
+        lse = np.empty((B, H, L), np.float64)
+        rc = self._lib.oracle_attn_partial(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                           _ptr(v, ctypes.c_float), _ptr(out, ctypes.c_double),
+                                           _ptr(lse, ctypes.c_double), B, H, L, d, scale, mk, w,
+                                           int(key_lo), int(key_hi))
+        if rc != 0:
+            raise RuntimeError(f"oracle_attn_partial failed ({rc})")
+        return out, lse
+
+
 def load_variant(path: str) -> Oracle:
     """Bind an Oracle to another compiled copy of the source (used by the tests
     that plant a mistake in a copy of the oracle and check that a pin fails)."""
@@ -184,3 +200,7 @@ def attention_kv_blockwise(*a, **kw):
 
 def attention_q_blockwise(*a, **kw):
     return _default().attention_q_blockwise(*a, **kw)
+
+
+def attention_partial(*a, **kw):
+    return _default().attention_partial(*a, **kw)

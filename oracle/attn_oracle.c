@@ -320,3 +320,50 @@ int oracle_attn_q_blockwise(const float* q, const float* k, const float* v,
   free(S);
   return 0;
 }
+
+/*
+ * The definition restricted to the keys j in [key_lo, key_hi): the partial
+ * result a key shard holds ([MOSAIC 2.1], before its tree reduction).  out is
+ * that range's softmax-weighted average of V (normalised within the range),
+ * lse its natural-log log-sum-exp; a row with no allowed key in the range gets
+ * out = 0 and lse = -inf.  One thread, plain loops.
+ */
+int oracle_attn_partial(const float* q, const float* k, const float* v, double* out,
+                        double* lse, int64_t B, int64_t H, int64_t L, int64_t d,
+                        double scale, int mask_kind, int64_t window, int64_t key_lo,
+                        int64_t key_hi) {
+  if (check_args(q, k, v, out, lse, B, H, L, d, mask_kind, window)) return -1;
+  if (key_lo < 0 || key_hi > L || key_hi < key_lo) return -1;
+  for (int64_t bh = 0; bh < B * H; ++bh) {
+    const float* kh = k + bh * L * d;
+    const float* vh = v + bh * L * d;
+    for (int64_t i = 0; i < L; ++i) {
+      const float* qi = q + (bh * L + i) * d;
+      double* o = out + (bh * L + i) * d;
+      double m = -INFINITY;
+      for (int64_t j = key_lo; j < key_hi; ++j) {
+        if (!allowed(i, j, mask_kind, window)) continue;
+        double dot = 0.0;
+        for (int64_t c = 0; c < d; ++c) dot += (double)qi[c] * (double)kh[j * d + c];
+        if (scale * dot > m) m = scale * dot;
+      }
+      for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+      if (m == -INFINITY) {
+        lse[bh * L + i] = -INFINITY;
+        continue;
+      }
+      double l = 0.0;
+      for (int64_t j = key_lo; j < key_hi; ++j) {
+        if (!allowed(i, j, mask_kind, window)) continue;
+        double dot = 0.0;
+        for (int64_t c = 0; c < d; ++c) dot += (double)qi[c] * (double)kh[j * d + c];
+        double p = exp(scale * dot - m);
+        l += p;
+        for (int64_t c = 0; c < d; ++c) o[c] += p * (double)vh[j * d + c];
+      }
+      for (int64_t c = 0; c < d; ++c) o[c] /= l;
+      lse[bh * L + i] = m + log(l);
+    }
+  }
+  return 0;
+}

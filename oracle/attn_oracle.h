@@ -75,6 +75,14 @@ int oracle_attn_q_blockwise(const float* q, const float* k, const float* v,
                             int64_t L, int64_t d, double scale, int mask_kind,
                             int64_t window, int64_t block);
 
+/* The definition restricted to keys [key_lo, key_hi) (a key shard's partial
+ * result, [MOSAIC 2.1]): out normalised within the range, lse over the range;
+ * rows with no allowed key in it get out = 0, lse = -inf. */
+int oracle_attn_partial(const float* q, const float* k, const float* v, double* out,
+                        double* lse, int64_t B, int64_t H, int64_t L, int64_t d,
+                        double scale, int mask_kind, int64_t window, int64_t key_lo,
+                        int64_t key_hi);
+
 #ifdef __cplusplus
 }
 #endif

@@ -305,6 +305,32 @@ def pin_rows_match(orc):
             assert l[n] == full_l[0, b_h, r]
 
 
+def pin_partials_merge_to_definition(orc):
+    """[MOSAIC 2.1]: partial results over disjoint key ranges combine into the
+    whole: LSE = ln sum_s e^LSE_s and O = sum_s e^(LSE_s - LSE) O_s.  Ranges
+    that hold no allowed key of a row give LSE_s = -inf (weight 0)."""
+    L, d = 45, 6
+    q, k, v = _rand((1, 2, L, d), 31), _rand((1, 2, L, d), 32), _rand((1, 2, L, d), 33)
+    for mask, window in (("none", 0), ("causal", 0), ("window", 4)):
+        full_o, full_l = orc.attention(q, k, v, mask=mask, window=window)
+        for bounds in ([0, 45], [0, 20, 45], [0, 1, 2, 44, 45], [0, 7, 14, 21, 28, 35, 45]):
+            parts = [orc.attention_partial(q, k, v, a, b, mask=mask, window=window)
+                     for a, b in zip(bounds[:-1], bounds[1:])]
+            lses = np.stack([p[1] for p in parts])
+            mx = lses.max(0)
+            w = np.exp(lses - mx)
+            lse = mx + np.log(w.sum(0))
+            o = sum(np.exp(p[1] - lse)[..., None] * p[0] for p in parts)
+            _close(lse, full_l, 1e-13, 1e-13, f"merged lse {mask} {bounds}")
+            _close(o, full_o, 1e-13, 1e-13, f"merged out {mask} {bounds}")
+    # an empty range is all -inf / 0
+    o, l = orc.attention_partial(q, k, v, 10, 10, mask="causal")
+    assert np.isneginf(l).all() and (o == 0).all()
+    # causal: row 3 has no allowed key in [20, 45)
+    o, l = orc.attention_partial(q, k, v, 20, 45, mask="causal")
+    assert np.isneginf(l[0, :, 3]).all() and (o[0, :, 3] == 0).all()
+
+
 ALL_PINS = [pin_brute_force, pin_golden, pin_kv_blockwise, pin_q_blockwise,
             pin_probability_rows, pin_identical_keys, pin_constant_v, pin_special_cases,
-            pin_overflow, pin_rows_match]
+            pin_overflow, pin_rows_match, pin_partials_merge_to_definition]
