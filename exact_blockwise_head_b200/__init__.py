@@ -28,6 +28,8 @@ ATTN_ERR_UNSUPPORTED = 2
 ATTN_ERR_MISALIGNED = 3
 ATTN_ERR_CUDA = 4
 ATTN_ERR_TIMEOUT = 5
+ATTN_ERR_SCRATCH_LIMIT = 6
+NOALLOC_SCRATCH_BYTES = 32 << 20  # ATTN_NOALLOC_SCRATCH_BYTES
 ATTN_DTYPE_BF16 = 0
 ATTN_DTYPE_F32 = 1
 
@@ -35,7 +37,7 @@ ATTN_DTYPE_F32 = 1
 EXPORTED = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ex", "attn_strerror", "attn_last_cuda_error",
             "attn_device_status", "attn_selftest_wait_timeout", "attn_kv_tile_range",
             "attn_kv_tile_class", "attn_kv_full_range", "attn_splitkv_workspace_bytes",
-            "attn_fwd_splitkv", "attn_merge", "attn_abi_version")
+            "attn_fwd_splitkv", "attn_merge", "attn_abi_version", "attn_fwd_splitkv_noalloc")
 
 
 class AttnParams(ctypes.Structure):
@@ -99,6 +101,7 @@ def _load():
             lib.attn_abi_version.argtypes = []
             lib.attn_splitkv_workspace_bytes.argtypes = [i, i, i, i, i]
             lib.attn_fwd_splitkv.argtypes = [ctypes.POINTER(AttnParams), i, vp, ctypes.c_size_t, vp]
+            lib.attn_fwd_splitkv_noalloc.argtypes = [ctypes.POINTER(AttnParams), i, vp]
             lib.attn_merge.argtypes = [vp, vp, i, ctypes.POINTER(i), i, i, vp, vp, i, i, i, i, i,
                                        vp]
             for name in EXPORTED:
@@ -230,6 +233,23 @@ def forward_splitkv(q, k, v, num_splits, scale=None, mask="none", window=0, bloc
                                       _stream_handle(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_splitkv")
+    return out, (lse if want_lse else None)
+
+
+def forward_splitkv_noalloc(q, k, v, num_splits, scale=None, mask="none", window=0,
+                            block_n=0, out=None, lse=None, want_lse=True, stream=None):
+    """forward_splitkv() with the partials in the library's fixed device scratch
+    (NOALLOC_SCRATCH_BYTES per device) instead of a workspace; the C call
+    allocates nothing (pass `out`/`lse` to keep this wrapper from allocating
+    them either).  Calls overlapping on one device share that scratch and race."""
+    import torch
+
+    p, out, lse = _params(q, k, v, scale, mask, window, block_n, out, lse, want_lse, 0)
+    with torch.cuda.device(q.device):
+        st = _load().attn_fwd_splitkv_noalloc(ctypes.byref(p), int(num_splits),
+                                              _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_splitkv_noalloc")
     return out, (lse if want_lse else None)
 
 

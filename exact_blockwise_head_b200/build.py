@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libebh_attn.so")
 TRACE_LIB = os.path.join(PKG, "libebh_attn_trace.so")
-SOURCES = ["api.cpp", "attn_sm100.cu", "attn_f32.cu", "attn_merge.cu"]
+SOURCES = ["api.cpp", "attn_sm100.cu", "attn_f32.cu", "attn_merge.cu", "noalloc.cu"]
 HEADERS = ["kernels.h", "sm100_ptx.cuh", "tiles.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

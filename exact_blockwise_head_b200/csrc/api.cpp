@@ -113,6 +113,10 @@ int check_device_sm100() {
 
 }  // namespace
 
+namespace ebh {
+void set_last_cuda_error(cudaError_t e) { g_last_cuda_error = static_cast<int>(e); }
+}  // namespace ebh
+
 extern "C" {
 
 int attn_fwd_ex(const attn_params* p, void* stream) {
@@ -174,6 +178,9 @@ const char* attn_strerror(int status) {
     case ATTN_ERR_MISALIGNED: return "misaligned pointer (q/k/v/out need 16 bytes, lse 4)";
     case ATTN_ERR_CUDA: return "CUDA runtime error (see attn_last_cuda_error)";
     case ATTN_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    case ATTN_ERR_SCRATCH_LIMIT:
+      return "problem needs more scratch than the fixed no-allocation scratch "
+             "(ATTN_NOALLOC_SCRATCH_BYTES) holds";
     default: return "unknown status";
   }
 }

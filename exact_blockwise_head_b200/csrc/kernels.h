@@ -53,4 +53,7 @@ int launch_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream, cudaErr
 int launch_merge(const MergeArgs& m, cudaStream_t stream, cudaError_t* err);
 int read_device_status(int device, int reset, cudaError_t* err);
 
+// Records e as this thread's attn_last_cuda_error() (defined in api.cpp).
+void set_last_cuda_error(cudaError_t e);
+
 }  // namespace ebh

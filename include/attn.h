@@ -72,7 +72,9 @@ enum {
   ATTN_ERR_MISALIGNED = 3,  /* q/k/v/out not 16-byte aligned, lse not 4-byte */
   ATTN_ERR_CUDA = 4,        /* a CUDA runtime call failed; attn_last_cuda_error()
                                gives its code */
-  ATTN_ERR_TIMEOUT = 5      /* a bounded wait inside a kernel ran out */
+  ATTN_ERR_TIMEOUT = 5,     /* a bounded wait inside a kernel ran out */
+  ATTN_ERR_SCRATCH_LIMIT = 6 /* the problem's partials do not fit the fixed
+                               scratch of attn_fwd_splitkv_noalloc */
 };
 
 /* Mask kinds. */
@@ -201,6 +203,38 @@ ATTN_API int attn_fwd_splitkv(const attn_params* p, int num_splits, void* worksp
 ATTN_API int attn_merge(const float* o_parts, const float* lse_parts, int num_splits,
                         const int* split_bounds, int mask_kind, int window, void* out,
                         float* lse, int out_dtype, int B, int H, int L, int d, void* stream);
+
+/*
+ * Split-KV forward with no workspace argument and no allocation.  The paper
+ * has no counterpart to this call: it is a library convenience for callers
+ * that cannot allocate device memory for attn_fwd_splitkv's workspace, such
+ * as code running under a host framework whose caching allocator owns all
+ * device memory, plugin interfaces that hand the library only its inputs and
+ * outputs, and latency-critical loops where cudaMalloc/cudaFree (which may
+ * synchronise the device) is not acceptable.
+ *
+ * It computes exactly what attn_fwd_splitkv computes, with the partials kept
+ * in a fixed scratch array of ATTN_NOALLOC_SCRATCH_BYTES that the library's
+ * device code carries on every device it is loaded on.  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *   - Limit: the partials of the runs actually used must fit, i.e.
+ *     attn_splitkv_workspace_bytes(B, H, L, d, runs) <= ATTN_NOALLOC_SCRATCH_BYTES
+ *     (at d=128 about 64K rows of B*H*L*runs); otherwise it returns
+ *     ATTN_ERR_SCRATCH_LIMIT and enqueues nothing.  With one run it is
+ *     attn_fwd_ex and the scratch is not touched.
+ *   - Set-up: the first call on a device (the current device) looks up the
+ *     scratch's device address with cudaGetSymbolAddress and keeps it; make
+ *     that first call before any stream capture on that device.  A failed
+ *     look-up returns ATTN_ERR_CUDA.
+ *   - Concurrency: every call on a device uses the same scratch, so calls
+ *     whose work may overlap on the GPU (unordered streams, several host
+ *     threads) race and corrupt each other's results; order them, e.g. on
+ *     one stream.
+ * Nothing in the scratch needs to start at zero.  Other arguments and errors
+ * as attn_fwd_splitkv.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+ATTN_API int attn_fwd_splitkv_noalloc(const attn_params* p, int num_splits, void* stream);
 
 /* ATTN_ABI_VERSION of the loaded library. */
 ATTN_API int attn_abi_version(void);
