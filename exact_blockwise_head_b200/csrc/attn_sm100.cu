@@ -17,20 +17,21 @@
 // Mapping onto Blackwell.  One persistent CTA per SM walks a static list of
 // work units; a unit is 256 query rows of one (batch, head), split into two
 // 128-row Q tiles that share the stream of K/V tiles.  Warp roles:
-//   warps 0-3   softmax for Q tile 0 (one thread per query row)
-//   warps 4-7   softmax for Q tile 1
-//   warp  8     TMA producer: Q tiles once per unit, then K_j, V_j into a ring
-//   warp  9     MMA issuer: S_t = Q_t K_j^T and O_t += P_t V_j (tcgen05, fp32
+//   warps 0-7   softmax for Q tile 0 (four threads per query row)
+//   warps 8-15  softmax for Q tile 1
+//   warp  16    TMA producer: Q tiles once per unit, then K_j, V_j into a ring
+//   warp  17    MMA issuer: S_t = Q_t K_j^T and O_t += P_t V_j (tcgen05, fp32
 //               accumulators in tensor memory); owns the tensor-memory block
-//   warps 10-11 idle
+//   warps 18-19 idle (they complete the producer / MMA warpgroup)
 // Tensor memory (columns): S_0 | S_1 | O_0 | O_1.  P_t (bf16, two per column)
 // is written over the first half of S_t and fed to the P.V product straight
 // from tensor memory.  The MMA warp interleaves the two Q tiles,
 //   S_0(j), P_1(j-1).V_(j-1), S_1(j), P_0(j).V_j, S_0(j+1), ...
-// so each softmax group works while the tensor core runs the other tile's
-// products.  Because tcgen05 MMAs complete in issue order, "S_t(j) done"
-// also means "P_t(j-1).V done", which lets the softmax thread rescale its
-// own row of O_t without any further barrier.
+// and the two softmax groups take turns at the exponentials, so that each
+// works while the tensor core runs the other tile's products.  Because
+// tcgen05 MMAs complete in issue order, "S_t(j) done" also means
+// "P_t(j-1).V done", which lets a softmax thread rescale its own rows of O_t
+// without any further barrier.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -83,7 +84,8 @@ enum : int {
   kEvEpilogue = 6, kEvEpilogueDone = 7,
   kEvKWait = 10, kEvKReady = 11, kEvVWait = 16, kEvVReady = 17,
   kEvPWait = 13, kEvPReady = 14,  // + 10 * Q tile
-  kEvSIssued = 30, kEvPVIssued = 32  // + Q tile
+  kEvSIssued = 30, kEvPVIssued = 32,  // + Q tile
+  kEvHalf1 = 40, kEvHalf2Loaded = 41, kEvHalf2 = 42, kEvRowMax = 43
 };
 #ifdef EBH_PIPELINE_TRACE
 constexpr int kTraceLen = 8192;
@@ -124,7 +126,8 @@ struct Cfg {
   static constexpr int kBarPFull = kBarSFull + kNQ;        // [kNQ]
   static constexpr int kBarOFull = kBarPFull + kNQ;        // [kNQ]
   static constexpr int kBarOEmpty = kBarOFull + kNQ;       // [kNQ]
-  static constexpr int kBarDrain = kBarOEmpty + kNQ;
+  static constexpr int kBarTok = kBarOEmpty + kNQ;        // [kNQ]
+  static constexpr int kBarDrain = kBarTok + kNQ;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kSmemBytes = 1024 + kSmemQ + kSmemKV + 8 * kNumBars + 16;
   static constexpr int kTmemNeed = 2 * BN + 2 * D;
@@ -221,6 +224,16 @@ __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
   }
   if (w.uhi <= w.ulo) w.ulo = w.uhi = 0;
   return w;
+}
+
+// The k-th unit of this CTA.  Units are dealt out in rounds of gridDim.x,
+// every other round in reverse CTA order: with causal units sorted longest
+// first, this evens the per-CTA totals (plain round-robin gives CTA 0 the
+// longest unit of every round).  Returns num_units once the CTA is done.
+__device__ __forceinline__ int unit_of(int k, const Params& p) {
+  const long long base = static_cast<long long>(k) * gridDim.x;
+  const long long u = base + ((k & 1) ? gridDim.x - 1 - blockIdx.x : blockIdx.x);
+  return u < p.num_units ? static_cast<int>(u) : p.num_units;
 }
 
 // Wait for all lanes of a warp; the outcome is made warp-uniform so that the
@@ -402,6 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(C::kBarPFull + t), kSoftmaxThreads);
       mbar_init(bar(C::kBarOFull + t), 1);
       mbar_init(bar(C::kBarOEmpty + t), kSoftmaxThreads);
+      mbar_init(bar(C::kBarTok + t), kSoftmaxWarps);
     }
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bar(C::kBarKVFull + s), 1);
@@ -440,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int kv_it = 0;
         int q_cnt[kNQ] = {0, 0};
         bool ok = true;
-        for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        for (int k = 0, u = unit_of(0, p); ok && u < p.num_units; u = unit_of(++k, p)) {
           const Unit w = decode_unit<BN>(u, p);
           auto load_q = [&](int t) -> bool {
             if (!w.valid[t]) return true;
@@ -535,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
 
-        for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        for (int k = 0, u = unit_of(0, p); ok && u < p.num_units; u = unit_of(++k, p)) {
           // key-block ranges of the two Q tiles (empty range: tile absent)
           int lo0, hi0, lo1, hi1;
           {
@@ -633,10 +647,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float cl2 = p.scale_log2;
     uint32_t phase = 0;  // bit 0: S_full parity, bit 1: O_full parity
     bool ok = true;
+    // The two Q tiles take turns at the exponentials: tile 1 starts key block
+    // j once tile 0 has finished its exponentials of block j, tile 0 starts
+    // block j once tile 1 has finished block j - 1.  Each tile counts the
+    // other's completions (one phase of kBarTok + tile per key block) to know
+    // which phase to wait for.  Without the turns, both groups share the
+    // exponential unit and finish together, and the tensor core then runs
+    // all four products of the step with no softmax to overlap.
+    const int other = t ^ 1;
+    uint32_t tok_base = 0;  // key blocks the other tile finished in earlier units
     EBH_TRACE_COUNTER;
 
-    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+    for (int k = 0, u = unit_of(0, p); ok && u < p.num_units; u = unit_of(++k, p)) {
       const TileWork w = decode_tile<BN>(u, t, p);
+      const TileWork wo = decode_tile<BN>(u, other, p);
+      const int o_lo = wo.valid ? wo.lo : 0, o_hi = wo.valid ? wo.hi : 0;
+      const uint32_t o_base = tok_base;
+      tok_base += static_cast<uint32_t>(o_hi - o_lo);
       if (!w.valid) continue;
       const int row_a = w.q_first + ra, row_b = w.q_first + rb;
       int full_lo, full_hi;  // key blocks that need no element mask
@@ -657,6 +684,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kHalf = BN / 16;  // column groups of 8 per half
         uint32_t sr[BN / 2];
         tmem_ld_half<BN>(tS, sr);
+        {
+          const int jo = t == 0 ? j - 1 : j;  // the other tile's block that goes first
+          if (jo >= o_lo && jo < o_hi) {
+            const uint32_t kt = o_base + static_cast<uint32_t>(jo - o_lo);
+            if (!(ok = warp_wait(bar(C::kBarTok + other), kt & 1, abort_flag, limit))) {
+              tmem_wait_ld();
+              break;
+            }
+          }
+        }
         tmem_wait_ld();
         reg_fence_half<BN>(sr);
         tmem_ld_half<BN>(tS + BN / 2, sr + BN / 4);
@@ -685,8 +722,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             probabilities<0, kHalf, false>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
           }
+          EBH_TRACE(kEvHalf1, j);
           tmem_wait_ld();
           reg_fence_half<BN>(sr + BN / 4);
+          EBH_TRACE(kEvHalf2Loaded, j);
           if (!full) mask_groups<kHalf, 2 * kHalf>(s, t0, a_lo, a_hi, b_lo, b_hi);
           if (full) {
             probabilities<kHalf, 2 * kHalf, kPolyOn>(s, cl2, m_a, m_b, tS, l_a, l_b,
@@ -694,10 +733,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             probabilities<kHalf, 2 * kHalf, false>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
           }
+          EBH_TRACE(kEvHalf2, j);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(C::kBarTok + t));
           float mta, mtb;
           row_max_pair<BN>(s, mta, mtb);
           mta *= cl2;
           mtb *= cl2;
+          EBH_TRACE(kEvRowMax, j);
           const bool grow_a = mta > m_a + kRescaleThreshold;
           const bool grow_b = mtb > m_b + kRescaleThreshold;
           if (__any_sync(0xffffffffu, grow_a || grow_b)) {
@@ -756,6 +799,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // that -inf - (-inf) never happens (its probabilities are all 0)
           probabilities<0, 2 * kHalf, false>(s, cl2, m_a == -INFINITY ? 0.f : m_a,
                                       m_b == -INFINITY ? 0.f : m_b, tS, l_a, l_b, lr_a, lr_b);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(C::kBarTok + t));
         }
         tmem_wait_st();
         tc_fence_before();
