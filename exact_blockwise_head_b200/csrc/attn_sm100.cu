@@ -450,7 +450,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_shrink<kOtherRegs>();
     if (warp == kProducerWarp) {
       // ------------------------------------------------------------ producer
-      if (lane == 0) {
+      // The whole warp walks the schedule (its counters stay warp-uniform);
+      // one elected lane issues the copies.
+      const bool leader = elect_one_sync();
+      {
         int kv_it = 0;
         int q_cnt[kNQ] = {0, 0};
         bool ok = true;
@@ -458,14 +461,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           const Unit w = decode_unit<BN>(u, p);
           auto load_q = [&](int t) -> bool {
             if (!w.valid[t]) return true;
-            if (!wait_bounded(bar(C::kBarQEmpty + t), (q_cnt[t] & 1) ^ 1, abort_flag, limit))
+            if (!warp_wait(bar(C::kBarQEmpty + t), (q_cnt[t] & 1) ^ 1, abort_flag, limit))
               return false;
-            mbar_arrive_expect_tx(bar(C::kBarQFull + t), C::kQTileBytes);
-            const uint32_t dst = smem_addr(sQ + t * C::kQTileBytes);
+            if (leader) {
+              mbar_arrive_expect_tx(bar(C::kBarQFull + t), C::kQTileBytes);
+              const uint32_t dst = smem_addr(sQ + t * C::kQTileBytes);
   #pragma unroll
-            for (int c = 0; c < C::kDChunks; ++c)
-              tma_load_3d(dst + c * kBM * 128, &tm_q, bar(C::kBarQFull + t), c * 64, w.q_first[t],
-                          w.bh);
+              for (int c = 0; c < C::kDChunks; ++c)
+                tma_load_3d(dst + c * kBM * 128, &tm_q, bar(C::kBarQFull + t), c * 64,
+                            w.q_first[t], w.bh);
+            }
+            __syncwarp();
             ++q_cnt[t];
             return true;
           };
@@ -474,15 +480,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
               const int s = kv_it % C::kStages;
-              ok = wait_bounded(bar(C::kBarKVEmpty + s), ((kv_it / C::kStages) & 1) ^ 1, abort_flag,
-                                limit);
+              ok = warp_wait(bar(C::kBarKVEmpty + s), ((kv_it / C::kStages) & 1) ^ 1, abort_flag,
+                             limit);
               if (!ok) break;
-              mbar_arrive_expect_tx(bar(C::kBarKVFull + s), C::kKVTileBytes);
-              const uint32_t dst = smem_addr(sKV + s * C::kKVTileBytes);
-              const CUtensorMap* map = which == 0 ? &tm_k : &tm_v;
+              if (leader) {
+                mbar_arrive_expect_tx(bar(C::kBarKVFull + s), C::kKVTileBytes);
+                const uint32_t dst = smem_addr(sKV + s * C::kKVTileBytes);
+                const CUtensorMap* map = which == 0 ? &tm_k : &tm_v;
   #pragma unroll
-              for (int c = 0; c < C::kDChunks; ++c)
-                tma_load_3d(dst + c * BN * 128, map, bar(C::kBarKVFull + s), c * 64, j * BN, w.bh);
+                for (int c = 0; c < C::kDChunks; ++c)
+                  tma_load_3d(dst + c * BN * 128, map, bar(C::kBarKVFull + s), c * 64, j * BN,
+                              w.bh);
+              }
+              __syncwarp();
               ++kv_it;
             }
           }
@@ -499,7 +509,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == kMmaWarp) {
       // ------------------------------------------------------------ MMA issuer
-      if (lane == 0) {
+      // The whole warp walks the schedule, so that counters and descriptors
+      // are warp-uniform (uniform registers); one elected lane issues each
+      // tcgen05 instruction, and the commits, which track the MMAs of the
+      // issuing thread.  With a single thread running the loop, every
+      // descriptor had to be moved into the uniform datapath per instruction.
+      const bool leader = elect_one_sync();
+      {
         constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, BN, false);
         constexpr uint32_t idesc_o = idesc_bf16_f32(kBM, D, true);
         constexpr uint32_t kStageUnits = C::kKVTileBytes >> 4;
@@ -523,28 +539,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a0 = lo_q + t * kQTileUnits;
           const uint32_t b0 = lo_k + kst * kStageUnits;
           const uint32_t d = tmem + C::kColS + t * BN;
+          if (leader) {
   #pragma unroll
-          for (int k = 0; k < D / 16; ++k)
-            mma_ss(d, desc(a0 + (((k / 4) * kBM * 128 + (k % 4) * 32) >> 4)),
-                   desc(b0 + (((k / 4) * BN * 128 + (k % 4) * 32) >> 4)), idesc_s,
-                   k > 0 ? 1u : 0u);
+            for (int k = 0; k < D / 16; ++k)
+              mma_ss(d, desc(a0 + (((k / 4) * kBM * 128 + (k % 4) * 32) >> 4)),
+                     desc(b0 + (((k / 4) * BN * 128 + (k % 4) * 32) >> 4)), idesc_s,
+                     k > 0 ? 1u : 0u);
+          }
+          __syncwarp();
+        };
+        auto commit = [&](uint32_t b) {
+          if (leader) mma_commit(b);
+          __syncwarp();
         };
         auto issue_pv = [&](int t, int vst, bool first) -> bool {
           EBH_TRACE(kEvPWait + 10 * t, 0);
-          if (!wait_bounded(bar(C::kBarPFull + t), (par_p >> t) & 1, abort_flag, limit))
+          if (!warp_wait(bar(C::kBarPFull + t), (par_p >> t) & 1, abort_flag, limit))
             return false;
           EBH_TRACE(kEvPReady + 10 * t, 0);
           par_p ^= 1u << t;
-          if (first && !wait_bounded(bar(C::kBarOEmpty + t), (par_oe >> t) & 1, abort_flag, limit))
+          if (first && !warp_wait(bar(C::kBarOEmpty + t), (par_oe >> t) & 1, abort_flag, limit))
             return false;
           tc_fence_after();
           const uint32_t b0 = lo_v + vst * kStageUnits;
           const uint32_t d = tmem + C::kColO + t * D;
           const uint32_t a = tmem + C::kColS + t * BN;
+          if (leader) {
   #pragma unroll
-          for (int k = 0; k < BN / 16; ++k)
-            mma_ts(d, a + k * 8, desc(b0 + ((k * 16 * 128) >> 4)), idesc_o,
-                   (first && k == 0) ? 0u : 1u);
+            for (int k = 0; k < BN / 16; ++k)
+              mma_ts(d, a + k * 8, desc(b0 + ((k * 16 * 128) >> 4)), idesc_o,
+                     (first && k == 0) ? 0u : 1u);
+          }
+          __syncwarp();
           EBH_TRACE(kEvPVIssued + t, 0);
           return true;
         };
@@ -569,53 +595,53 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t vph = ((kv_it + 1) / C::kStages) & 1;
             kv_it += 2;
             EBH_TRACE(kEvKWait, j);
-            if (!(ok = wait_bounded(bar(C::kBarKVFull + kst), kph, abort_flag, limit))) break;
+            if (!(ok = warp_wait(bar(C::kBarKVFull + kst), kph, abort_flag, limit))) break;
             EBH_TRACE(kEvKReady, j);
             const bool in0 = j >= lo0 && j < hi0, in1 = j >= lo1 && j < hi1;
             if (in0) {
-              if (j == lo0 && !(ok = wait_bounded(bar(C::kBarQFull + 0), par_q & 1, abort_flag,
+              if (j == lo0 && !(ok = warp_wait(bar(C::kBarQFull + 0), par_q & 1, abort_flag,
                                                   limit)))
                 break;
               tc_fence_after();
               issue_s(0, kst);
               EBH_TRACE(kEvSIssued + 0, j);
-              mma_commit(bar(C::kBarSFull + 0));
-              if (j == hi0 - 1) mma_commit(bar(C::kBarQEmpty + 0));
+              commit(bar(C::kBarSFull + 0));
+              if (j == hi0 - 1) commit(bar(C::kBarQEmpty + 0));
             }
             if (pend_v >= 0) {
               if (!(ok = issue_pv(1, pend_v, j - 1 == lo1))) break;
-              mma_commit(bar(C::kBarKVEmpty + pend_v));
-              if (j - 1 == hi1 - 1) mma_commit(bar(C::kBarOFull + 1));
+              commit(bar(C::kBarKVEmpty + pend_v));
+              if (j - 1 == hi1 - 1) commit(bar(C::kBarOFull + 1));
               pend_v = -1;
             }
             if (in1) {
-              if (j == lo1 && !(ok = wait_bounded(bar(C::kBarQFull + 1), (par_q >> 1) & 1,
+              if (j == lo1 && !(ok = warp_wait(bar(C::kBarQFull + 1), (par_q >> 1) & 1,
                                                   abort_flag, limit)))
                 break;
               tc_fence_after();
               issue_s(1, kst);
               EBH_TRACE(kEvSIssued + 1, j);
-              mma_commit(bar(C::kBarSFull + 1));
-              if (j == hi1 - 1) mma_commit(bar(C::kBarQEmpty + 1));
+              commit(bar(C::kBarSFull + 1));
+              if (j == hi1 - 1) commit(bar(C::kBarQEmpty + 1));
             }
-            mma_commit(bar(C::kBarKVEmpty + kst));  // K_j no longer needed
+            commit(bar(C::kBarKVEmpty + kst));  // K_j no longer needed
             EBH_TRACE(kEvVWait, j);
-            if (!(ok = wait_bounded(bar(C::kBarKVFull + vst), vph, abort_flag, limit))) break;
+            if (!(ok = warp_wait(bar(C::kBarKVFull + vst), vph, abort_flag, limit))) break;
             EBH_TRACE(kEvVReady, j);
             if (in0) {
               if (!(ok = issue_pv(0, vst, j == lo0))) break;
-              if (j == hi0 - 1) mma_commit(bar(C::kBarOFull + 0));
+              if (j == hi0 - 1) commit(bar(C::kBarOFull + 0));
             }
             if (in1) {
               pend_v = vst;
             } else {
-              mma_commit(bar(C::kBarKVEmpty + vst));
+              commit(bar(C::kBarKVEmpty + vst));
             }
           }
           if (ok && pend_v >= 0) {
             if ((ok = issue_pv(1, pend_v, uhi - 1 == lo1))) {
-              mma_commit(bar(C::kBarKVEmpty + pend_v));
-              if (uhi - 1 == hi1 - 1) mma_commit(bar(C::kBarOFull + 1));
+              commit(bar(C::kBarKVEmpty + pend_v));
+              if (uhi - 1 == hi1 - 1) commit(bar(C::kBarOFull + 1));
             }
           }
           // Q tiles and O accumulators used by this unit move to their next phase
@@ -624,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           par_oe ^= used;
         }
         // No MMA may still be writing tensor memory when it is freed.
-        mma_commit(bar(C::kBarDrain));
+        commit(bar(C::kBarDrain));
         drain_wait(bar(C::kBarDrain), 0, limit);
       }
     }
