@@ -62,12 +62,14 @@ static_assert(kSoftmaxRegs * kNQ * kSoftmaxThreads + kOtherRegs * 128 <= kLaunch
 // Tuning knobs of the softmax arithmetic.  kPolyEvery: one column group of
 // eight in kPolyEvery takes its exponentials from a polynomial on the FMA pipe
 // instead of the MUFU pipe (tiles without masked elements only; 0 = none).
-// kScalarMath: scalar fp32 FMA/add instead of the paired f32x2 forms.
+// kScalarMath: scalar fp32 FMA/add (default) instead of the paired f32x2
+// forms; the paired forms need register-pair moves on the half-rate ALU pipe
+// that cost more than the FMA-pipe slots they save.
 #ifndef EBH_POLY_EVERY
 #define EBH_POLY_EVERY 0
 #endif
 #ifndef EBH_SCALAR_MATH
-#define EBH_SCALAR_MATH 0
+#define EBH_SCALAR_MATH 1
 #endif
 constexpr int kPolyEvery = EBH_POLY_EVERY > 0 ? EBH_POLY_EVERY : 1;
 constexpr bool kPolyOn = EBH_POLY_EVERY > 0;
