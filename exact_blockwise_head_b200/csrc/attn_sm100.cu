@@ -125,8 +125,8 @@ struct Cfg {
   static constexpr int kBarKVFull = kBarQEmpty + kNQ;  // [kStages]
   static constexpr int kBarKVEmpty = kBarKVFull + kStages;
   static constexpr int kBarSFull = kBarKVEmpty + kStages;  // [kNQ]
-  static constexpr int kBarPFull = kBarSFull + kNQ;        // [kNQ]
-  static constexpr int kBarOFull = kBarPFull + kNQ;        // [kNQ]
+  static constexpr int kBarPFull = kBarSFull + kNQ;        // [kNQ][2]: halves of P_t
+  static constexpr int kBarOFull = kBarPFull + 2 * kNQ;    // [kNQ]
   static constexpr int kBarOEmpty = kBarOFull + kNQ;       // [kNQ]
   static constexpr int kBarTok = kBarOEmpty + kNQ;        // [kNQ]
   static constexpr int kBarDrain = kBarTok + kNQ;
@@ -371,6 +371,36 @@ __device__ __forceinline__ void probabilities(const float* s, float cl2, float m
   }
 }
 
+// Same as probabilities(), but the packed bf16 pairs stay in registers
+// (pk[2 (m - G0) + {0, 1}]) for a later store_p().
+template <int G0, int G1>
+__device__ __forceinline__ void probabilities_regs(const float* s, float cl2, float ma, float mb,
+                                                   uint32_t* pk, float& l_a, float& l_b,
+                                                   float& lr_a, float& lr_b) {
+#pragma unroll
+  for (int m = G0; m < G1; ++m) {
+    const float p0 = ex2_approx(fmaf(s[4 * m], cl2, -ma));
+    const float p1 = ex2_approx(fmaf(s[4 * m + 1], cl2, -ma));
+    const float p2 = ex2_approx(fmaf(s[4 * m + 2], cl2, -mb));
+    const float p3 = ex2_approx(fmaf(s[4 * m + 3], cl2, -mb));
+    const uint32_t a = pack_bf16x2(p0, p1), b = pack_bf16x2(p2, p3);
+    pk[2 * (m - G0)] = a;
+    pk[2 * (m - G0) + 1] = b;
+    l_a += p0;
+    l_b += p2;
+    l_a += p1;
+    l_b += p3;
+    acc_bf16x2_sum(lr_a, a);
+    acc_bf16x2_sum(lr_b, b);
+  }
+}
+// Store the packed pairs of column groups [G0, G1) (multiples of 4).
+template <int G0, int G1>
+__device__ __forceinline__ void store_p(uint32_t tS, const uint32_t* pk) {
+#pragma unroll
+  for (int ch = G0 / 4; ch < G1 / 4; ++ch) tmem_st_16x128b_x4(tS + 16 * ch, pk + 8 * (ch - G0 / 4));
+}
+
 // O rows *= alpha (alpha_a for the thread's first row, alpha_b for its
 // second), all D columns, through tensor memory.  The caller guarantees no MMA
 // is writing O_t (its previous P.V product was issued before the S_t product
@@ -414,7 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(C::kBarQFull + t), 1);
       mbar_init(bar(C::kBarQEmpty + t), 1);
       mbar_init(bar(C::kBarSFull + t), 1);
-      mbar_init(bar(C::kBarPFull + t), kSoftmaxThreads);
+      mbar_init(bar(C::kBarPFull + 2 * t), kSoftmaxThreads);
+      mbar_init(bar(C::kBarPFull + 2 * t + 1), kSoftmaxThreads);
       mbar_init(bar(C::kBarOFull + t), 1);
       mbar_init(bar(C::kBarOEmpty + t), kSoftmaxThreads);
       mbar_init(bar(C::kBarTok + t), kSoftmaxWarps);
@@ -554,25 +585,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (leader) mma_commit(b);
           __syncwarp();
         };
+        // O_t (+)= P_t V_j in two halves of the keys: each half is issued as
+        // soon as the softmax group has released that half of P_t.
         auto issue_pv = [&](int t, int vst, bool first) -> bool {
-          EBH_TRACE(kEvPWait + 10 * t, 0);
-          if (!warp_wait(bar(C::kBarPFull + t), (par_p >> t) & 1, abort_flag, limit))
-            return false;
-          EBH_TRACE(kEvPReady + 10 * t, 0);
-          par_p ^= 1u << t;
-          if (first && !warp_wait(bar(C::kBarOEmpty + t), (par_oe >> t) & 1, abort_flag, limit))
-            return false;
-          tc_fence_after();
           const uint32_t b0 = lo_v + vst * kStageUnits;
           const uint32_t d = tmem + C::kColO + t * D;
           const uint32_t a = tmem + C::kColS + t * BN;
-          if (leader) {
   #pragma unroll
-            for (int k = 0; k < BN / 16; ++k)
-              mma_ts(d, a + k * 8, desc(b0 + ((k * 16 * 128) >> 4)), idesc_o,
-                     (first && k == 0) ? 0u : 1u);
+          for (int h = 0; h < 2; ++h) {
+            EBH_TRACE(kEvPWait + 10 * t, h);
+            if (!warp_wait(bar(C::kBarPFull + 2 * t + h), (par_p >> t) & 1, abort_flag, limit))
+              return false;
+            EBH_TRACE(kEvPReady + 10 * t, h);
+            if (h == 0 && first &&
+                !warp_wait(bar(C::kBarOEmpty + t), (par_oe >> t) & 1, abort_flag, limit))
+              return false;
+            tc_fence_after();
+            if (leader) {
+  #pragma unroll
+              for (int k = h * (BN / 32); k < (h + 1) * (BN / 32); ++k)
+                mma_ts(d, a + k * 8, desc(b0 + ((k * 16 * 128) >> 4)), idesc_o,
+                       (first && k == 0) ? 0u : 1u);
+            }
+            __syncwarp();
           }
-          __syncwarp();
+          par_p ^= 1u << t;
           EBH_TRACE(kEvPVIssued + t, 0);
           return true;
         };
@@ -739,6 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // The branch must be warp-uniform: both sides run warp-collective
         // tensor-memory instructions and shuffles.
+        bool released_a = false;  // first half of P already handed to the MMA warp
         if (__all_sync(0xffffffffu, m_a != -INFINITY && m_b != -INFINITY)) {
           // Speculate that the stale reference max still holds (the tile max
           // exceeds it by at most the threshold): the exponentials need not
@@ -755,15 +793,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           reg_fence_half<BN>(sr + BN / 4);
           EBH_TRACE(kEvHalf2Loaded, j);
           if (!full) mask_groups<kHalf, 2 * kHalf>(s, t0, a_lo, a_hi, b_lo, b_hi);
-          if (full) {
-            probabilities<kHalf, 2 * kHalf, kPolyOn>(s, cl2, m_a, m_b, tS, l_a, l_b,
-                                                               lr_a, lr_b);
-          } else {
-            probabilities<kHalf, 2 * kHalf, false>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
-          }
-          EBH_TRACE(kEvHalf2, j);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(C::kBarTok + t));
           float mta, mtb;
           row_max_pair<BN>(s, mta, mtb);
           mta *= cl2;
@@ -771,7 +800,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           EBH_TRACE(kEvRowMax, j);
           const bool grow_a = mta > m_a + kRescaleThreshold;
           const bool grow_b = mtb > m_b + kRescaleThreshold;
-          if (__any_sync(0xffffffffu, grow_a || grow_b)) {
+          if (!__any_sync(0xffffffffu, grow_a || grow_b)) {
+            // The speculation held.  Second half into registers; by then the
+            // first half's stores have landed, so it is handed to the MMA
+            // warp at once and its P.V product overlaps the second half's
+            // stores.
+            uint32_t pk2[BN / 8];
+            probabilities_regs<kHalf, 2 * kHalf>(s, cl2, m_a, m_b, pk2, l_a, l_b, lr_a, lr_b);
+            EBH_TRACE(kEvHalf2, j);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::kBarTok + t));
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(C::kBarPFull + 2 * t));
+            released_a = true;
+            store_p<kHalf, 2 * kHalf>(tS, pk2);
+          } else {
             // rare: redo the tile against the grown maximum
             float alpha_a = 1.f, alpha_b = 1.f;
             if (grow_a) {
@@ -788,6 +832,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             lr_b = lr_b0 * alpha_b;
             rescale_o_rows<D>(tO, alpha_a, alpha_b);
             probabilities<0, 2 * kHalf, false>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
+            EBH_TRACE(kEvHalf2, j);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::kBarTok + t));
           }
         } else {
           // first key block with an allowed key for some row of this thread:
@@ -833,7 +880,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         EBH_TRACE(kEvPWritten, j);
-        mbar_arrive(bar(C::kBarPFull + t));
+        if (!released_a) mbar_arrive(bar(C::kBarPFull + 2 * t));
+        mbar_arrive(bar(C::kBarPFull + 2 * t + 1));
       }
       if (!ok) break;
 
