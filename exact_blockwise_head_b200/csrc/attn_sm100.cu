@@ -904,6 +904,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool ok_a = row_a < p.L, ok_b = row_b < p.L;
       const float lse_a = l_a > 0.f ? (m_a + log2f(l_a)) * 0.69314718055994531f : -INFINITY;
       const float lse_b = l_b > 0.f ? (m_b + log2f(l_b)) * 0.69314718055994531f : -INFINITY;
+      // All of O_t's rows of this thread in one load; once it has landed the
+      // accumulator is free for the next unit's first P.V product.
+      uint32_t o[D / 2];
+      if constexpr (D == 128) {
+        tmem_ld_16x256b_x16(tO, o);
+        tmem_wait_ld();
+        reg_fence64(o);
+      } else {
+        tmem_ld_16x256b_x8(tO, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarOEmpty + t));
+      // register 4m + {0, 1}: row a, columns 8m + 2 t0 + {0, 1}; 4m + {2, 3}: row b
       if (p.o_part == nullptr) {
         uint32_t* dst_a = reinterpret_cast<uint32_t*>(
             static_cast<uint16_t*>(p.out) +
@@ -911,22 +926,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t* dst_b = reinterpret_cast<uint32_t*>(
             static_cast<uint16_t*>(p.out) +
             (static_cast<size_t>(w.bh) * p.L + (ok_b ? row_b : 0)) * D);
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[16];
-          tmem_ld_16x256b_x4(tO + 32 * c, o);
-          tmem_wait_ld();
-          reg_fence16(o);
 #pragma unroll
-          for (int mm = 0; mm < 4; ++mm) {
-            const int col2 = (32 * c + 8 * mm + 2 * t0) / 2;  // pair index in the row
-            const uint32_t va = pack_bf16x2(__uint_as_float(o[4 * mm]) * inv_a,
-                                            __uint_as_float(o[4 * mm + 1]) * inv_a);
-            const uint32_t vb = pack_bf16x2(__uint_as_float(o[4 * mm + 2]) * inv_b,
-                                            __uint_as_float(o[4 * mm + 3]) * inv_b);
-            if (ok_a) dst_a[col2] = va;
-            if (ok_b) dst_b[col2] = vb;
-          }
+        for (int m = 0; m < D / 8; ++m) {
+          const int col2 = 4 * m + t0;  // pair index in the row
+          const uint32_t va = pack_bf16x2(__uint_as_float(o[4 * m]) * inv_a,
+                                          __uint_as_float(o[4 * m + 1]) * inv_a);
+          const uint32_t vb = pack_bf16x2(__uint_as_float(o[4 * m + 2]) * inv_b,
+                                          __uint_as_float(o[4 * m + 3]) * inv_b);
+          if (ok_a) dst_a[col2] = va;
+          if (ok_b) dst_b[col2] = vb;
         }
         if (t0 == 0 && p.lse != nullptr) {
           if (ok_a) p.lse[static_cast<size_t>(w.bh) * p.L + row_a] = lse_a;
@@ -939,31 +947,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             p.o_part + (head * p.L + (ok_a ? row_a : 0)) * D);
         float2* dst_b = reinterpret_cast<float2*>(
             p.o_part + (head * p.L + (ok_b ? row_b : 0)) * D);
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[16];
-          tmem_ld_16x256b_x4(tO + 32 * c, o);
-          tmem_wait_ld();
-          reg_fence16(o);
 #pragma unroll
-          for (int mm = 0; mm < 4; ++mm) {
-            const int col2 = (32 * c + 8 * mm + 2 * t0) / 2;
-            if (ok_a)
-              dst_a[col2] = make_float2(__uint_as_float(o[4 * mm]) * inv_a,
-                                        __uint_as_float(o[4 * mm + 1]) * inv_a);
-            if (ok_b)
-              dst_b[col2] = make_float2(__uint_as_float(o[4 * mm + 2]) * inv_b,
-                                        __uint_as_float(o[4 * mm + 3]) * inv_b);
-          }
+        for (int m = 0; m < D / 8; ++m) {
+          const int col2 = 4 * m + t0;
+          if (ok_a)
+            dst_a[col2] = make_float2(__uint_as_float(o[4 * m]) * inv_a,
+                                      __uint_as_float(o[4 * m + 1]) * inv_a);
+          if (ok_b)
+            dst_b[col2] = make_float2(__uint_as_float(o[4 * m + 2]) * inv_b,
+                                      __uint_as_float(o[4 * m + 3]) * inv_b);
         }
         if (t0 == 0) {
           if (ok_a) p.lse_part[head * p.L + row_a] = lse_a;
           if (ok_b) p.lse_part[head * p.L + row_b] = lse_b;
         }
       }
-      tc_fence_before();
       EBH_TRACE(kEvEpilogueDone, 0);
-      mbar_arrive(bar(C::kBarOEmpty + t));
     }
   }
 
