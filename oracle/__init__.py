@@ -24,7 +24,7 @@ _LIB = os.path.join(_HERE, "_attn_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-MASKS = {"none": 0, "causal": 1, "window": 2}
+MASKS = {"none": 0, "causal": 1, "window": 2, "causal_window": 3}
 
 
 def build(force: bool = False) -> str:

@@ -29,6 +29,7 @@
 static int allowed(int64_t i, int64_t j, int mask_kind, int64_t window) {
   if (mask_kind == ORACLE_MASK_CAUSAL) return j <= i;
   if (mask_kind == ORACLE_MASK_WINDOW) return (i - j <= window) && (j - i <= window);
+  if (mask_kind == ORACLE_MASK_CAUSAL_WINDOW) return (j <= i) && (i - j <= window);
   return 1;
 }
 
@@ -37,8 +38,9 @@ static int check_args(const float* q, const float* k, const float* v,
                       int64_t L, int64_t d, int mask_kind, int64_t window) {
   if (!q || !k || !v || !out || !lse) return -1;
   if (B <= 0 || H <= 0 || L <= 0 || d <= 0) return -1;
-  if (mask_kind < ORACLE_MASK_NONE || mask_kind > ORACLE_MASK_WINDOW) return -1;
-  if (mask_kind == ORACLE_MASK_WINDOW && window < 0) return -1;
+  if (mask_kind < ORACLE_MASK_NONE || mask_kind > ORACLE_MASK_CAUSAL_WINDOW) return -1;
+  if ((mask_kind == ORACLE_MASK_WINDOW || mask_kind == ORACLE_MASK_CAUSAL_WINDOW) && window < 0)
+    return -1;
   return 0;
 }
 

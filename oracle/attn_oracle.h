@@ -43,7 +43,10 @@ extern "C" {
 enum {
   ORACLE_MASK_NONE = 0,   /* every key */
   ORACLE_MASK_CAUSAL = 1, /* key j <= query i */
-  ORACLE_MASK_WINDOW = 2  /* |i - j| <= window */
+  ORACLE_MASK_WINDOW = 2, /* |i - j| <= window */
+  /* i - window <= j <= i: the band of [LONGSEQ] section 2.1 kept on the
+   * causal side only (the page's tril(w).triu(-w) with tril at diagonal 0) */
+  ORACLE_MASK_CAUSAL_WINDOW = 3
 };
 
 /* The plain definition, one query row at a time, rows spread over nthreads. */

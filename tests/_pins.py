@@ -34,7 +34,8 @@ GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 # --------------------------------------------------------------------------
 def dense_mask(L, mask, window):
     """0/1 matrix: causal is tril(diagonal=0); window is tril(diagonal=w) times
-    triu(diagonal=-w) as [LONGSEQ 2.1] builds it."""
+    triu(diagonal=-w) as [LONGSEQ 2.1] builds it; causal_window is that band
+    with its upper side at the diagonal, tril(diagonal=0) times triu(diagonal=-w)."""
     M = [[1] * L for _ in range(L)]
     for i in range(L):
         for j in range(L):
@@ -42,6 +43,10 @@ def dense_mask(L, mask, window):
                 M[i][j] = 1 if j - i <= 0 else 0
             elif mask == "window":
                 tril = 1 if j - i <= window else 0
+                triu = 1 if j - i >= -window else 0
+                M[i][j] = tril * triu
+            elif mask == "causal_window":
+                tril = 1 if j - i <= 0 else 0
                 triu = 1 if j - i >= -window else 0
                 M[i][j] = tril * triu
     return M
@@ -91,7 +96,7 @@ def pin_brute_force(orc):
     seed = 100
     for L, d in cases:
         for mask, window in (("none", 0), ("causal", 0), ("window", 0), ("window", 1),
-                             ("window", 3)):
+                             ("window", 3), ("causal_window", 0), ("causal_window", 2)):
             seed += 1
             q = _rand((1, 1, L, d), seed)
             k = _rand((1, 1, L, d), seed + 1000)
@@ -140,7 +145,7 @@ def pin_kv_blockwise(orc):
     definition for every block size 1..L, and for large blocks at L=512."""
     L, d = 40, 6
     q, k, v = _rand((1, 2, L, d), 1), _rand((1, 2, L, d), 2), _rand((1, 2, L, d), 3)
-    for mask, window in (("none", 0), ("causal", 0), ("window", 4)):
+    for mask, window in (("none", 0), ("causal", 0), ("window", 4), ("causal_window", 6)):
         ref = orc.attention(q, k, v, mask=mask, window=window)
         for block in range(1, L + 1):
             got = orc.attention_kv_blockwise(q, k, v, block, mask=mask, window=window)
@@ -148,7 +153,7 @@ def pin_kv_blockwise(orc):
             _close(got[1], ref[1], 1e-12, 1e-13, f"kv-blockwise lse b={block} {mask}")
     L, d = 512, 16
     q, k, v = _rand((1, 1, L, d), 4), _rand((1, 1, L, d), 5), _rand((1, 1, L, d), 6)
-    for mask, window in (("none", 0), ("causal", 0), ("window", 37)):
+    for mask, window in (("none", 0), ("causal", 0), ("window", 37), ("causal_window", 100)):
         ref = orc.attention(q, k, v, mask=mask, window=window)
         for block in (1, 7, 64, 128, 256, 1000):
             got = orc.attention_kv_blockwise(q, k, v, block, mask=mask, window=window)
@@ -161,7 +166,7 @@ def pin_q_blockwise(orc):
     unblocked result for every block size."""
     L, d = 29, 5
     q, k, v = _rand((2, 1, L, d), 7), _rand((2, 1, L, d), 8), _rand((2, 1, L, d), 9)
-    for mask, window in (("none", 0), ("causal", 0), ("window", 2)):
+    for mask, window in (("none", 0), ("causal", 0), ("window", 2), ("causal_window", 3)):
         ref = orc.attention(q, k, v, mask=mask, window=window)
         for block in list(range(1, L + 2)) + [256]:
             got = orc.attention_q_blockwise(q, k, v, block, mask=mask, window=window)
@@ -187,7 +192,7 @@ def pin_probability_rows(orc):
     """Probability rows sum to 1, are >= 0, and are exactly 0 on masked keys."""
     L, d = 24, 4
     q, k = _rand((1, 2, L, d), 10, 2.0), _rand((1, 2, L, d), 11, 2.0)
-    for mask, window in (("none", 0), ("causal", 0), ("window", 3)):
+    for mask, window in (("none", 0), ("causal", 0), ("window", 3), ("causal_window", 4)):
         P, _ = _probabilities(orc, q, k, 0.5, mask, window)
         M = np.array(dense_mask(L, mask, window), bool)
         assert (P >= 0).all()
@@ -205,8 +210,8 @@ def pin_identical_keys(orc):
     v = _rand((1, 1, L, d), 14)
     scale = 0.7
     M_all = {m: np.array(dense_mask(L, m, w), bool) for m, w in
-             (("none", 0), ("causal", 0), ("window", 5))}
-    for mask, window in (("none", 0), ("causal", 0), ("window", 5)):
+             (("none", 0), ("causal", 0), ("window", 5), ("causal_window", 7))}
+    for mask, window in (("none", 0), ("causal", 0), ("window", 5), ("causal_window", 7)):
         out, lse = orc.attention(q, k, v, scale=scale, mask=mask, window=window)
         M = M_all[mask]
         for i in range(L):
@@ -222,7 +227,7 @@ def pin_constant_v(orc):
     q, k = _rand((2, 2, L, d), 15, 3.0), _rand((2, 2, L, d), 16, 3.0)
     c = _rand((1, 1, 1, d), 17)
     v = np.broadcast_to(c, (2, 2, L, d)).copy()
-    for mask, window in (("none", 0), ("causal", 0), ("window", 6)):
+    for mask, window in (("none", 0), ("causal", 0), ("window", 6), ("causal_window", 6)):
         out, _ = orc.attention(q, k, v, mask=mask, window=window)
         _close(out, np.broadcast_to(c.astype(np.float64), out.shape), 1e-14, 1e-14,
                f"constant V {mask}")
@@ -247,8 +252,17 @@ def pin_special_cases(orc):
     out, lse = orc.attention(q, k, v, scale=scale, mask="causal")
     _close(out[0, 0, 0], v[0, 0, 0].astype(np.float64), 0.0, 0.0, "causal row 0")
     _close(lse[0, 0, 0], s_ii[0, 0, 0], 1e-15, 0.0, "causal row 0 lse")
+    # the causal side of the band: w=0 keeps only the diagonal, w >= L-1 is causal
+    out, lse = orc.attention(q, k, v, scale=scale, mask="causal_window", window=0)
+    _close(out, v.astype(np.float64), 1e-15, 0.0, "causal w=0 -> V")
+    _close(lse, s_ii, 1e-14, 1e-15, "causal w=0 -> lse = s_ii")
+    ref_c = orc.attention(q, k, v, scale=scale, mask="causal")
+    for w in (L - 1, L, 10 * L):
+        got = orc.attention(q, k, v, scale=scale, mask="causal_window", window=w)
+        _close(got[0], ref_c[0], 0.0, 0.0, f"causal w={w} -> causal")
+        _close(got[1], ref_c[1], 0.0, 0.0, f"causal w={w} -> causal lse")
     zq = np.zeros_like(q)
-    for mask, window in (("none", 0), ("causal", 0), ("window", 3)):
+    for mask, window in (("none", 0), ("causal", 0), ("window", 3), ("causal_window", 4)):
         out, lse = orc.attention(zq, k, v, scale=scale, mask=mask, window=window)
         M = np.array(dense_mask(L, mask, window), bool)
         for i in range(L):
@@ -278,7 +292,7 @@ def pin_overflow(orc):
     k, v = _rand((1, 2, L, d), 25), _rand((1, 2, L, d), 26)
     for mult in (8.0, 64.0, 1000.0):
         q = _rand((1, 2, L, d), 27, mult)
-        for mask, window in (("none", 0), ("causal", 0), ("window", 9)):
+        for mask, window in (("none", 0), ("causal", 0), ("window", 9), ("causal_window", 9)):
             out, lse = orc.attention(q, k, v, mask=mask, window=window)
             assert np.isfinite(out).all() and np.isfinite(lse).all(), (mult, mask)
             M = np.array(dense_mask(L, mask, window), bool)
@@ -295,7 +309,7 @@ def pin_rows_match(orc):
     """The selected-rows call returns the same rows as the whole-problem call."""
     B, H, L, d = 1, 3, 70, 8
     q, k, v = _rand((B, H, L, d), 28), _rand((B, H, L, d), 29), _rand((B, H, L, d), 30)
-    for mask, window in (("none", 0), ("causal", 0), ("window", 11)):
+    for mask, window in (("none", 0), ("causal", 0), ("window", 11), ("causal_window", 11)):
         full_o, full_l = orc.attention(q, k, v, mask=mask, window=window)
         bh = [0, 0, 1, 2, 2, 2]
         rows = [0, 69, 5, 0, 34, 69]
@@ -311,7 +325,7 @@ def pin_partials_merge_to_definition(orc):
     that hold no allowed key of a row give LSE_s = -inf (weight 0)."""
     L, d = 45, 6
     q, k, v = _rand((1, 2, L, d), 31), _rand((1, 2, L, d), 32), _rand((1, 2, L, d), 33)
-    for mask, window in (("none", 0), ("causal", 0), ("window", 4)):
+    for mask, window in (("none", 0), ("causal", 0), ("window", 4), ("causal_window", 9)):
         full_o, full_l = orc.attention(q, k, v, mask=mask, window=window)
         for bounds in ([0, 45], [0, 20, 45], [0, 1, 2, 44, 45], [0, 7, 14, 21, 28, 35, 45]):
             parts = [orc.attention_partial(q, k, v, a, b, mask=mask, window=window)

@@ -33,6 +33,8 @@ MUTANTS = [
     ("kv_sum_not_rescaled", "l *= alpha;", ""),
     ("q_block_tail_dropped", "int64_t i1 = i0 + block < L ? i0 + block : L;",
      "int64_t i1 = i0 + block < L ? i0 + block : L - 1;"),
+    ("causal_window_two_sided", "(j <= i) && (i - j <= window)", "(i - j <= window)"),
+    ("causal_window_off_by_one", "(j <= i) && (i - j <= window)", "(j <= i) && (i - j < window)"),
     ("partial_not_normalised", "for (int64_t c = 0; c < d; ++c) o[c] /= l;\n      lse[bh * L + i]",
      "lse[bh * L + i]"),
     ("partial_range_shifted", "for (int64_t j = key_lo; j < key_hi; ++j) {\n        if (!allowed(i, j, mask_kind, window)) continue;\n        double dot = 0.0;\n        for (int64_t c = 0; c < d; ++c) dot += (double)qi[c] * (double)kh[j * d + c];\n        double p",
