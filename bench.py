@@ -68,6 +68,9 @@ def allowed_pairs(L: int, mask: str, window: int) -> int:
     if mask == "causal":
         return L * (L + 1) // 2
     w = min(window, L - 1)
+    if mask == "causal_window":
+        # row i sees keys [max(0, i-w), i]: w+1 keys, fewer for rows 0..w-1
+        return L * (w + 1) - w * (w + 1) // 2
     # row i sees keys [max(0, i-w), min(L-1, i+w)]
     total = L * (2 * w + 1)
     total -= w * (w + 1)  # clipped at the left edge (rows 0..w-1) and the right edge
@@ -407,7 +410,7 @@ def main():
     if rank == 0 and not args.no_sweep and world == 1:
         others = [n for n in ("mha_bf16_L2048_d64", "mha_bf16_L2048_d64_qx8",
                               "window512_bf16_L32768_d128", "causal_bf16_L131072_d128",
-                              "causal_bf16_L8192_d128")
+                              "causal_window1024_bf16_L32768_d128", "causal_bf16_L8192_d128")
                   if n != w.name]
         del qe, ke, ve
         line["other_workloads_kernel_only"] = sweep_other(ebh, torch, others)

@@ -24,6 +24,11 @@ int fail_cuda(cudaError_t e) {
   return ATTN_ERR_CUDA;
 }
 
+// Mask kinds that read `window`.
+bool has_window(int mask_kind) {
+  return mask_kind == ATTN_MASK_WINDOW || mask_kind == ATTN_MASK_CAUSAL_WINDOW;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Half-open byte ranges [a, a + na) and [b, b + nb) overlap?
@@ -41,9 +46,9 @@ int validate(const attn_params* p, ebh::FwdArgs* out) {
   if (static_cast<long long>(p->B) * p->H > 0x7fffffffLL) return ATTN_ERR_INVALID;
   if (!std::isfinite(p->scale) || !(p->scale > 0.f)) return ATTN_ERR_INVALID;
   if (p->mask_kind != ATTN_MASK_NONE && p->mask_kind != ATTN_MASK_CAUSAL &&
-      p->mask_kind != ATTN_MASK_WINDOW)
+      p->mask_kind != ATTN_MASK_WINDOW && p->mask_kind != ATTN_MASK_CAUSAL_WINDOW)
     return ATTN_ERR_INVALID;
-  if (p->mask_kind == ATTN_MASK_WINDOW && p->window < 0) return ATTN_ERR_INVALID;
+  if (has_window(p->mask_kind) && p->window < 0) return ATTN_ERR_INVALID;
   if (p->dtype == ATTN_DTYPE_BF16) {
     if (p->block_n != 0 && p->block_n != 64 && p->block_n != 128) return ATTN_ERR_INVALID;
   } else if (p->block_n != 0) {
@@ -83,7 +88,7 @@ int validate(const attn_params* p, ebh::FwdArgs* out) {
   out->scale = p->scale;
   out->mask_kind = p->mask_kind;
   // a band at least L wide allows every pair: clamp so index sums stay small
-  out->window = p->mask_kind == ATTN_MASK_WINDOW ? (p->window > p->L ? p->L : p->window) : 0;
+  out->window = has_window(p->mask_kind) ? (p->window > p->L ? p->L : p->window) : 0;
   out->block_n = p->dtype == ATTN_DTYPE_BF16 ? (p->block_n == 0 ? 128 : p->block_n) : 0;
   out->timeout_ns = p->wait_timeout_ns ? p->wait_timeout_ns : kDefaultTimeoutNs;
   return ATTN_OK;
@@ -208,8 +213,8 @@ int attn_kv_tile_range(int L, int q_first, int q_last, int mask_kind, int window
                        int* lo, int* hi) {
   if (!lo || !hi || L <= 0 || block_n <= 0 || q_first < 0 || q_last < q_first || q_last >= L)
     return ATTN_ERR_INVALID;
-  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_WINDOW) return ATTN_ERR_INVALID;
-  if (mask_kind == ATTN_MASK_WINDOW && window < 0) return ATTN_ERR_INVALID;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_CAUSAL_WINDOW) return ATTN_ERR_INVALID;
+  if (has_window(mask_kind) && window < 0) return ATTN_ERR_INVALID;
   ebh::kv_tile_range(L, q_first, q_last, mask_kind, window, block_n, *lo, *hi);
   return ATTN_OK;
 }
@@ -218,8 +223,8 @@ int attn_kv_tile_class(int L, int q_first, int q_last, int j, int mask_kind, int
                        int block_n) {
   if (L <= 0 || block_n <= 0 || q_first < 0 || q_last < q_first || q_last >= L)
     return -ATTN_ERR_INVALID;
-  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_WINDOW) return -ATTN_ERR_INVALID;
-  if (mask_kind == ATTN_MASK_WINDOW && window < 0) return -ATTN_ERR_INVALID;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_CAUSAL_WINDOW) return -ATTN_ERR_INVALID;
+  if (has_window(mask_kind) && window < 0) return -ATTN_ERR_INVALID;
   return ebh::kv_tile_class(L, q_first, q_last, j, mask_kind, window, block_n);
 }
 
@@ -296,8 +301,8 @@ int attn_merge(const float* o_parts, const float* lse_parts, int num_splits,
   if (num_splits < 1 || num_splits > ebh::kMaxSplits) return ATTN_ERR_INVALID;
   if (B <= 0 || H <= 0 || L <= 0) return ATTN_ERR_INVALID;
   if (static_cast<long long>(B) * H > 0x7fffffffLL) return ATTN_ERR_INVALID;
-  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_WINDOW) return ATTN_ERR_INVALID;
-  if (mask_kind == ATTN_MASK_WINDOW && window < 0) return ATTN_ERR_INVALID;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_CAUSAL_WINDOW) return ATTN_ERR_INVALID;
+  if (has_window(mask_kind) && window < 0) return ATTN_ERR_INVALID;
   if (out_dtype != ATTN_DTYPE_BF16 && out_dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (split_bounds[0] != 0) return ATTN_ERR_INVALID;
@@ -321,7 +326,7 @@ int attn_merge(const float* o_parts, const float* lse_parts, int num_splits,
   m.L = L;
   m.d = d;
   m.mask_kind = mask_kind;
-  m.window = mask_kind == ATTN_MASK_WINDOW ? (window > L ? L : window) : 0;
+  m.window = has_window(mask_kind) ? (window > L ? L : window) : 0;
   cudaError_t err = cudaSuccess;
   st = ebh::launch_merge(m, static_cast<cudaStream_t>(stream), &err);
   if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
@@ -332,8 +337,8 @@ int attn_kv_full_range(int L, int q_first, int q_last, int mask_kind, int window
                        int* lo, int* hi) {
   if (!lo || !hi || L <= 0 || block_n <= 0 || q_first < 0 || q_last < q_first || q_last >= L)
     return ATTN_ERR_INVALID;
-  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_WINDOW) return ATTN_ERR_INVALID;
-  if (mask_kind == ATTN_MASK_WINDOW && window < 0) return ATTN_ERR_INVALID;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_CAUSAL_WINDOW) return ATTN_ERR_INVALID;
+  if (has_window(mask_kind) && window < 0) return ATTN_ERR_INVALID;
   ebh::kv_full_range(L, q_first, q_last, mask_kind, window, block_n, *lo, *hi);
   return ATTN_OK;
 }

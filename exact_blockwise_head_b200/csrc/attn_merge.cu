@@ -39,6 +39,9 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Merg
   } else if (m.mask_kind == kMaskWindow) {
     kmin = (long long)i - m.window > 0 ? (long long)i - m.window : 0;
     kmax = (long long)i + m.window < m.L - 1 ? (long long)i + m.window : m.L - 1;
+  } else if (m.mask_kind == kMaskCausalWindow) {
+    kmin = (long long)i - m.window > 0 ? (long long)i - m.window : 0;
+    kmax = i;
   }
   auto contributes = [&](int s) {
     const long long lo = m.bounds[s] > kmin ? m.bounds[s] : kmin;

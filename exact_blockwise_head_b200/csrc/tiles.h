@@ -4,8 +4,9 @@
 //
 // Masks: causal keeps key j <= query i; window keeps |i - j| <= w, the band of
 // "Attention optimisation strategies and practice for long-sequence inference"
-// (trdm.cn), section 2.1.  Skipping blocks with no allowed pair is what makes
-// the window cost O(L w) instead of O(L^2), the point of that section.
+// (trdm.cn), section 2.1; causal window keeps that band's causal side only,
+// i - w <= j <= i.  Skipping blocks with no allowed pair is what makes the
+// windows cost O(L w) instead of O(L^2), the point of that section.
 #pragma once
 
 #ifdef __CUDACC__
@@ -16,7 +17,7 @@
 
 namespace ebh {
 
-enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskWindow = 2 };
+enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskWindow = 2, kMaskCausalWindow = 3 };
 enum : int { kTileEmpty = 0, kTilePartial = 1, kTileFull = 2 };
 
 // Key blocks [lo, hi) holding at least one allowed key for some query row in
@@ -35,6 +36,11 @@ EBH_HD void kv_tile_range(int L, int q_first, int q_last, int mask_kind,
     const long long b = (long long)q_last + window;
     const long long h = b / bn + 1;
     hi = h < nkv ? (int)h : nkv;
+  } else if (mask_kind == kMaskCausalWindow) {
+    const long long a = (long long)q_first - window;
+    lo = a <= 0 ? 0 : (int)(a / bn);
+    const int h = q_last / bn + 1;
+    hi = h < nkv ? h : nkv;
   }
 }
 
@@ -56,6 +62,11 @@ EBH_HD int kv_tile_class(int L, int q_first, int q_last, int j, int mask_kind,
       return kTileFull;
     return kTilePartial;
   }
+  if (mask_kind == kMaskCausalWindow) {
+    if (k0 > q_last || k1 < (long long)q_first - window) return kTileEmpty;
+    if (k1 < L && k1 <= q_first && (long long)q_last - k0 <= window) return kTileFull;
+    return kTilePartial;
+  }
   return k1 < L ? kTileFull : kTilePartial;
 }
 
@@ -75,6 +86,12 @@ EBH_HD void kv_full_range(int L, int q_first, int q_last, int mask_kind, int win
     if (a > 0) lo = (a + bn - 1) / bn;
     const long long h = ((long long)q_first + window + 1) / bn;
     if (h < hi) hi = h;
+  } else if (mask_kind == kMaskCausalWindow) {
+    // q_last - j bn <= w  and  (j + 1) bn - 1 <= q_first
+    const long long a = (long long)q_last - window;
+    if (a > 0) lo = (a + bn - 1) / bn;
+    const long long h = ((long long)q_first + 1) / bn;
+    if (h < hi) hi = h;
   }
   if (hi < lo) hi = lo;
   flo = (int)lo;
@@ -93,6 +110,11 @@ EBH_HD void row_allowed_cols(int L, int i, int j, int mask_kind, int window,
     if (h < hi) hi = h;
   } else if (mask_kind == kMaskWindow) {
     const long long h = (long long)i + window - k0 + 1;
+    if (h < hi) hi = h;
+    const long long l = (long long)i - window - k0;
+    if (l > lo) lo = l;
+  } else if (mask_kind == kMaskCausalWindow) {
+    const long long h = (long long)i - k0 + 1;
     if (h < hi) hi = h;
     const long long l = (long long)i - window - k0;
     if (l > lo) lo = l;

@@ -18,7 +18,7 @@ from dataclasses import dataclass, replace
 
 import torch
 
-MASK_KINDS = {"none": 0, "causal": 1, "window": 2}
+MASK_KINDS = {"none": 0, "causal": 1, "window": 2, "causal_window": 3}
 
 
 @dataclass(frozen=True)
@@ -44,7 +44,8 @@ class Workload:
         return replace(self, **kw)
 
 
-# The five workloads of the pages' problem statement, by what they are.
+# The five workloads of the pages' problem statement, by what they are, and
+# the one-sided window workload of the next row.
 WORKLOADS = {
     # tiny exact attention, fp32
     "tiny_f32_L256_d64": Workload("tiny_f32_L256_d64", 1, 2, 256, 64, dtype="f32"),
@@ -62,6 +63,11 @@ WORKLOADS = {
     # long-sequence causal attention at L=131072
     "causal_bf16_L131072_d128": Workload("causal_bf16_L131072_d128", 1, 8, 131072, 128,
                                          mask="causal"),
+    # one-sided (causal) sliding window i-1024 <= j <= i at L=32768: as many
+    # keys per row as the two-sided +-512 band
+    "causal_window1024_bf16_L32768_d128": Workload("causal_window1024_bf16_L32768_d128", 1,
+                                                   32, 32768, 128, mask="causal_window",
+                                                   window=1024),
 }
 
 

@@ -22,6 +22,8 @@
  *   ATTN_MASK_WINDOW  |i - j| <= window, the band of "Attention optimisation
  *                     strategies and practice for long-sequence inference"
  *                     (trdm.cn), section 2.1, applied additively (-inf)
+ *   ATTN_MASK_CAUSAL_WINDOW
+ *                     i - window <= j <= i: that band's causal side only
  * Every mask allows the diagonal, so no row is ever fully masked.
  *
  * Layout.  q, k, v, out are dense row-major [B, H, L, d] arrays (d fastest,
@@ -78,7 +80,7 @@ enum {
 };
 
 /* Mask kinds. */
-enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1, ATTN_MASK_WINDOW = 2 };
+enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1, ATTN_MASK_WINDOW = 2, ATTN_MASK_CAUSAL_WINDOW = 3 };
 
 /* Element types. */
 enum { ATTN_DTYPE_BF16 = 0, ATTN_DTYPE_F32 = 1 };
@@ -93,7 +95,7 @@ enum { ATTN_TILE_EMPTY = 0, ATTN_TILE_PARTIAL = 1, ATTN_TILE_FULL = 2 };
  * softmax runs in fp32 with exp2; the probabilities are rounded to bf16 for
  * the P.V product; out is rounded to bf16 (nearest-even).  B, H, L >= 1 with
  * B*H <= 2^31-1; scale finite and > 0 (the pages use 1/sqrt(d)); window >= 0,
- * read only for ATTN_MASK_WINDOW.  Keys are visited in blocks of 128.
+ * read only for the two window masks.  Keys are visited in blocks of 128.
  */
 ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
              int B, int H, int L, int d, float scale, int mask_kind, int window,

@@ -74,7 +74,8 @@ BAD = [
     ("scale inf", dict(scale=float("inf")), ebh.ATTN_ERR_INVALID),
     ("scale 0", dict(scale=0.0), ebh.ATTN_ERR_INVALID),
     ("scale<0", dict(scale=-1.0), ebh.ATTN_ERR_INVALID),
-    ("mask 3", dict(mask_kind=3), ebh.ATTN_ERR_INVALID),
+    ("mask 4", dict(mask_kind=4), ebh.ATTN_ERR_INVALID),
+    ("causal window<0", dict(mask_kind=3, window=-1), ebh.ATTN_ERR_INVALID),
     ("mask -1", dict(mask_kind=-1), ebh.ATTN_ERR_INVALID),
     ("window<0", dict(mask_kind=2, window=-1), ebh.ATTN_ERR_INVALID),
     ("block_n 96", dict(block_n=96), ebh.ATTN_ERR_INVALID),

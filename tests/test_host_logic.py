@@ -16,7 +16,9 @@ from tests._pins import dense_mask
 
 @pytest.mark.parametrize("L", [1, 2, 3, 10, 64, 129])
 @pytest.mark.parametrize("mask,window", [("none", 0), ("causal", 0), ("window", 0),
-                                         ("window", 1), ("window", 7), ("window", 500)])
+                                         ("window", 1), ("window", 7), ("window", 500),
+                                         ("causal_window", 0), ("causal_window", 1),
+                                         ("causal_window", 7), ("causal_window", 500)])
 def test_allowed_pairs_closed_forms(L, mask, window):
     assert bench.allowed_pairs(L, mask, window) == int(np.array(dense_mask(L, mask, window)).sum())
 

@@ -16,7 +16,8 @@ def _gpu():
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("mask,window", [("none", 0), ("causal", 0), ("window", 40)])
+@pytest.mark.parametrize("mask,window", [("none", 0), ("causal", 0), ("window", 40),
+                                         ("causal_window", 40)])
 def test_constant_values_pass_through(d, mask, window):
     q, k, _ = G.rand_qkv(1, 2, 777, d, seed=1, q_mult=3.0)
     c = torch.randn(d, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
@@ -25,7 +26,8 @@ def test_constant_values_pass_through(d, mask, window):
     assert np.abs(out - c.double().numpy()).max() <= G.BF16_OUT_ATOL
 
 
-@pytest.mark.parametrize("mask,window", [("none", 0), ("causal", 0), ("window", 9)])
+@pytest.mark.parametrize("mask,window", [("none", 0), ("causal", 0), ("window", 9),
+                                         ("causal_window", 9)])
 def test_identical_keys_average_the_allowed_values(mask, window):
     L, d = 300, 64
     q, _, v = G.rand_qkv(1, 1, L, d, seed=3)
@@ -44,6 +46,17 @@ def test_window_zero_returns_v():
     q, k, v = G.rand_qkv(1, 2, 500, 128, seed=5)
     out, _ = G.gpu_forward(q, k, v, mask="window", window=0)
     assert np.array_equal(out, v.double().numpy())
+
+
+def test_causal_window_zero_returns_v_and_wide_equals_causal():
+    q, k, v = G.rand_qkv(1, 2, 450, 128, seed=7)
+    out, _ = G.gpu_forward(q, k, v, mask="causal_window", window=0)
+    assert np.array_equal(out, v.double().numpy())
+    a = G.gpu_forward(q, k, v, mask="causal")
+    for w in (449, 450, 10 ** 6):
+        b = G.gpu_forward(q, k, v, mask="causal_window", window=w)
+        assert np.abs(a[0] - b[0]).max() <= G.BF16_OUT_ATOL
+        assert np.abs(a[1] - b[1]).max() <= G.BF16_LSE_ATOL
 
 
 def test_wide_window_equals_no_mask():

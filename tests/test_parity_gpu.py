@@ -32,7 +32,8 @@ def test_fp32_tiny_exact_attention():
 
 @pytest.mark.parametrize("L,d,mask,window", [
     (1, 64, "none", 0), (33, 17, "causal", 0), (100, 128, "window", 7),
-    (257, 256, "causal", 0), (300, 1, "window", 0), (129, 96, "none", 0)])
+    (257, 256, "causal", 0), (300, 1, "window", 0), (129, 96, "none", 0),
+    (150, 64, "causal_window", 9), (70, 3, "causal_window", 0)])
 def test_fp32_ragged(L, d, mask, window):
     q, k, v = G.rand_qkv(2, 1, L, d, seed=L + d, dtype="f32")
     out, lse = G.gpu_forward(q, k, v, mask=mask, window=window)
@@ -47,7 +48,7 @@ SMALL = [
     (1, 1, 1025, 64), (1, 1, 2125, 128),
 ]
 MASKS = [("none", 0), ("causal", 0), ("window", 0), ("window", 5), ("window", 128),
-         ("window", 300)]
+         ("window", 300), ("causal_window", 0), ("causal_window", 5), ("causal_window", 200)]
 
 
 @pytest.mark.parametrize("shape", SMALL, ids=lambda s: "B{}H{}L{}d{}".format(*s))
@@ -73,7 +74,7 @@ def test_bf16_scale_argument(d):
 def test_bf16_many_heads_persistent_schedule():
     """More work units than SMs, so every CTA walks several units."""
     q, k, v = G.rand_qkv(3, 37, 600, 64, seed=11)
-    for mask, window in (("causal", 0), ("window", 100), ("none", 0)):
+    for mask, window in (("causal", 0), ("window", 100), ("none", 0), ("causal_window", 77)):
         out, lse = G.gpu_forward(q, k, v, mask=mask, window=window)
         ref_o, ref_l = G.oracle_full(q, k, v, mask=mask, window=window)
         G.check_bf16(out, lse, ref_o, ref_l, f"many heads {mask}")
@@ -112,6 +113,10 @@ def test_full_causal_L8192_block_sizes_agree():
 
 def test_full_window512_L32768():
     _sampled(ebh.WORKLOADS["window512_bf16_L32768_d128"])
+
+
+def test_full_causal_window1024_L32768():
+    _sampled(ebh.WORKLOADS["causal_window1024_bf16_L32768_d128"])
 
 
 def test_full_causal_L131072_O_of_L_memory():

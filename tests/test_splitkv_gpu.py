@@ -39,6 +39,8 @@ CASES = [
     ((1, 3, 700, 64), "none", 0, 64),
     ((1, 1, 1, 128), "causal", 0, 3),
     ((1, 2, 777, 128), "window", 0, 3),
+    ((1, 2, 1500, 128), "causal_window", 300, 5),
+    ((2, 1, 900, 64), "causal_window", 0, 3),
     ((2, 2, 1500, 64), "causal", 0, 7),
 ]
 
@@ -57,7 +59,7 @@ def test_merge_of_oracle_partials():
     B, H, L, d = 1, 2, 900, 128
     q, k, v = G.rand_qkv(B, H, L, d, seed=77)
     qf, kf, vf = (G.as_f32(t) for t in (q, k, v))
-    for mask, window in (("none", 0), ("causal", 0), ("window", 50)):
+    for mask, window in (("none", 0), ("causal", 0), ("window", 50), ("causal_window", 60)):
         bounds = [0, 100, 333, 334, 900]
         parts = [oracle.attention_partial(qf, kf, vf, a, b, mask=mask, window=window)
                  for a, b in zip(bounds[:-1], bounds[1:])]

@@ -22,7 +22,9 @@ def _dense(L, mask, window):
 CASES = []
 for L in (1, 2, 63, 64, 65, 127, 128, 129, 200, 256, 300):
     for mask, window in (("none", 0), ("causal", 0), ("window", 0), ("window", 1),
-                         ("window", 63), ("window", 64), ("window", 130), ("window", 1000)):
+                         ("window", 63), ("window", 64), ("window", 130), ("window", 1000),
+                         ("causal_window", 0), ("causal_window", 1), ("causal_window", 63),
+                         ("causal_window", 64), ("causal_window", 130), ("causal_window", 1000)):
         CASES.append((L, mask, window))
 
 
