@@ -37,7 +37,8 @@ ATTN_DTYPE_F32 = 1
 EXPORTED = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ex", "attn_strerror", "attn_last_cuda_error",
             "attn_device_status", "attn_selftest_wait_timeout", "attn_kv_tile_range",
             "attn_kv_tile_class", "attn_kv_full_range", "attn_splitkv_workspace_bytes",
-            "attn_fwd_splitkv", "attn_merge", "attn_abi_version", "attn_fwd_splitkv_noalloc")
+            "attn_fwd_splitkv", "attn_merge", "attn_abi_version", "attn_fwd_splitkv_noalloc",
+            "attn_fwd_rows", "attn_seq_unshard")
 
 
 class AttnParams(ctypes.Structure):
@@ -102,6 +103,8 @@ def _load():
             lib.attn_splitkv_workspace_bytes.argtypes = [i, i, i, i, i]
             lib.attn_fwd_splitkv.argtypes = [ctypes.POINTER(AttnParams), i, vp, ctypes.c_size_t, vp]
             lib.attn_fwd_splitkv_noalloc.argtypes = [ctypes.POINTER(AttnParams), i, vp]
+            lib.attn_fwd_rows.argtypes = [ctypes.POINTER(AttnParams), i, i, vp]
+            lib.attn_seq_unshard.argtypes = [vp, vp, i, i, i, i, i, i, vp]
             lib.attn_merge.argtypes = [vp, vp, i, ctypes.POINTER(i), i, i, vp, vp, i, i, i, i, i,
                                        vp]
             for name in EXPORTED:
@@ -131,7 +134,8 @@ def forward(q, k, v, scale=None, mask="none", window=0, block_n=0, out=None, lse
 
     q, k, v: CUDA tensors of one shape [B, H, L, d], all bf16 (tensor-core path,
     d in {64, 128}) or all fp32 (CUDA-core path, d <= 256), contiguous.
-    mask: "none", "causal" (key j <= query i) or "window" (|i - j| <= window).
+    mask: "none", "causal" (key j <= query i), "window" (|i - j| <= window) or
+    "causal_window" (i - window <= j <= i).
     scale defaults to 1/sqrt(d).  Returns (out, lse); lse is None when
     want_lse is False.  The work is enqueued on `stream` (default: the current
     stream) and the call returns without synchronising.
@@ -171,6 +175,69 @@ def forward(q, k, v, scale=None, mask="none", window=0, block_n=0, out=None, lse
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_ex")
     return out, (lse if want_lse else None)
+
+
+def forward_rows(q, k, v, q_offset, scale=None, mask="none", window=0, block_n=0, out=None,
+                 lse=None, want_lse=True, stream=None):
+    """forward() for query rows placed inside a longer key sequence: q is
+    [B, H, Lq, d], k and v are [B, H, Lk, d], and query row i sits at key
+    position q_offset + i (0 <= q_offset, q_offset + Lq <= Lk).  Returns
+    (out [B, H, Lq, d], lse [B, H, Lq])."""
+    import torch
+
+    if q.dim() != 4 or k.shape != v.shape or q.shape[:2] != k.shape[:2] or q.shape[3] != k.shape[3]:
+        raise ValueError("q must be [B, H, Lq, d] and k, v [B, H, Lk, d]")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if mask not in MASK_KINDS:
+        raise ValueError(f"mask must be one of {sorted(MASK_KINDS)}")
+    if out is None:
+        out = torch.empty_like(q)
+    if want_lse and lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    p = AttnParams()
+    p.dtype = ATTN_DTYPE_BF16 if q.dtype == torch.bfloat16 else ATTN_DTYPE_F32
+    p.q, p.k, p.v, p.out = q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr()
+    p.lse = lse.data_ptr() if (want_lse and lse is not None) else None
+    p.B, p.H, p.L, p.d = B, H, Lq, d
+    p.scale = float(scale)
+    p.mask_kind = MASK_KINDS[mask]
+    p.window = int(window)
+    p.block_n = int(block_n)
+    p.wait_timeout_ns = 0
+    with torch.cuda.device(q.device):
+        st = _load().attn_fwd_rows(ctypes.byref(p), int(Lk), int(q_offset),
+                                   _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_rows")
+    return out, (lse if want_lse else None)
+
+
+def seq_unshard(gathered, out=None, stream=None):
+    """[S, B, H, Ls, d] rank-major shards (an all-gather's result) ->
+    [B, H, S*Ls, d], shard g's row c at key g*Ls + c."""
+    import torch
+
+    if gathered.dim() != 5 or not gathered.is_cuda or not gathered.is_contiguous():
+        raise ValueError("gathered must be a contiguous CUDA tensor [S, B, H, Ls, d]")
+    if gathered.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("gathered must be bf16 or fp32")
+    S, B, H, Ls, d = gathered.shape
+    if out is None:
+        out = torch.empty((B, H, S * Ls, d), dtype=gathered.dtype, device=gathered.device)
+    with torch.cuda.device(gathered.device):
+        st = _load().attn_seq_unshard(gathered.data_ptr(), out.data_ptr(), S, B, H, Ls, d,
+                                      gathered.element_size(), _stream_handle(stream, gathered.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_seq_unshard")
+    return out
 
 
 def _params(q, k, v, scale, mask, window, block_n, out, lse, want_lse, wait_timeout_ns):

@@ -137,6 +137,53 @@ int attn_fwd_ex(const attn_params* p, void* stream) {
   return st;
 }
 
+int attn_fwd_rows(const attn_params* p, int kv_len, int q_offset, void* stream) {
+  if (p == nullptr) return ATTN_ERR_INVALID;
+  if (kv_len <= 0 || q_offset < 0 || p->L <= 0 ||
+      static_cast<long long>(q_offset) + p->L > kv_len)
+    return ATTN_ERR_INVALID;
+  ebh::FwdArgs a;
+  int st = validate(p, &a);
+  if (st != ATTN_OK) return st;
+  {  // k and v hold kv_len rows: check the outputs against their full extent
+    const uint64_t elem = p->dtype == ATTN_DTYPE_BF16 ? 2 : 4;
+    const uint64_t kv_bytes = static_cast<uint64_t>(p->B) * p->H * kv_len * p->d * elem;
+    const uint64_t o_bytes = static_cast<uint64_t>(p->B) * p->H * p->L * p->d * elem;
+    const uint64_t l_bytes = static_cast<uint64_t>(p->B) * p->H * p->L * 4;
+    if (overlap(p->out, o_bytes, p->k, kv_bytes) || overlap(p->out, o_bytes, p->v, kv_bytes) ||
+        (p->lse && (overlap(p->lse, l_bytes, p->k, kv_bytes) ||
+                    overlap(p->lse, l_bytes, p->v, kv_bytes))))
+      return ATTN_ERR_INVALID;
+  }
+  a.Lk = kv_len;
+  a.q_shift = q_offset;
+  // the band is measured in key positions: clamp it to the keys, not the rows
+  a.window = has_window(p->mask_kind) ? (p->window > kv_len ? kv_len : p->window) : 0;
+  if ((st = check_device_sm100()) != ATTN_OK) return st;
+  cudaError_t err = cudaSuccess;
+  st = p->dtype == ATTN_DTYPE_BF16
+           ? ebh::launch_fwd_bf16_sm100(a, static_cast<cudaStream_t>(stream), &err)
+           : ebh::launch_fwd_f32(a, static_cast<cudaStream_t>(stream), &err);
+  if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
+  return st;
+}
+
+int attn_seq_unshard(const void* gathered, void* out, int S, int B, int H, int Ls, int d,
+                     int elem_bytes, void* stream) {
+  if (!gathered || !out || S <= 0 || B <= 0 || H <= 0 || Ls <= 0 || d <= 0) return ATTN_ERR_INVALID;
+  if (elem_bytes != 2 && elem_bytes != 4) return ATTN_ERR_INVALID;
+  if (static_cast<long long>(B) * H > 0x7fffffffLL ||
+      static_cast<long long>(S) * Ls > 0x7fffffffLL)
+    return ATTN_ERR_INVALID;
+  const uint64_t bytes = static_cast<uint64_t>(S) * B * H * Ls * d * elem_bytes;
+  if (overlap(gathered, bytes, out, bytes)) return ATTN_ERR_INVALID;
+  cudaError_t err = cudaSuccess;
+  const int st = ebh::launch_unshard(gathered, out, S, B * H, Ls, d, elem_bytes,
+                                     static_cast<cudaStream_t>(stream), &err);
+  if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
+  return st;
+}
+
 int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
              int L, int d, float scale, int mask_kind, int window, void* stream) {
   attn_params p = {};

@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(kThreadsF32)
     attn_fwd_f32_kernel(const float* __restrict__ q, const float* __restrict__ k,
                         const float* __restrict__ v, float* __restrict__ out,
                         float* __restrict__ lse, int L, int d, float scale, int mask_kind,
-                        int window) {
+                        int window, int Lk, int q_shift) {
   constexpr int DP = kParts * DPT;
   extern __shared__ float sm[];
   float* Ks = sm;                   // [kKeyTile][DP]
@@ -47,7 +47,8 @@ __global__ void __launch_bounds__(kThreadsF32)
   const int r = threadIdx.x / kParts;
   const int part = threadIdx.x % kParts;
   const int row = q_first + r;
-  const size_t head = static_cast<size_t>(bh) * L * d;
+  const size_t head = static_cast<size_t>(bh) * L * d;      // q, out: L rows per head
+  const size_t head_kv = static_cast<size_t>(bh) * Lk * d;  // k, v: Lk rows per head
 
   // this thread's slice of q: elements part, part + 4, part + 8, ...
   float qv[DPT], o[DPT];
@@ -60,21 +61,22 @@ __global__ void __launch_bounds__(kThreadsF32)
   float m = -INFINITY, l = 0.f;
 
   int lo, hi;
-  kv_tile_range(L, q_first, q_last, mask_kind, window, kKeyTile, lo, hi);
+  // query row r sits at key position r + q_shift
+  kv_tile_range(Lk, q_first + q_shift, q_last + q_shift, mask_kind, window, kKeyTile, lo, hi);
   for (int jt = lo; jt < hi; ++jt) {
     __syncthreads();
     for (int e = threadIdx.x; e < kKeyTile * DP; e += kThreadsF32) {
       const int kr = e / DP, c = e % DP;
       const int key = jt * kKeyTile + kr;
-      const bool in = key < L && c < d;
-      const size_t off = head + static_cast<size_t>(in ? key : 0) * d + (in ? c : 0);
+      const bool in = key < Lk && c < d;
+      const size_t off = head_kv + static_cast<size_t>(in ? key : 0) * d + (in ? c : 0);
       Ks[e] = in ? k[off] : 0.f;
       Vs[e] = in ? v[off] : 0.f;
     }
     __syncthreads();
 
     int c_lo, c_hi;
-    row_allowed_cols(L, row, jt, mask_kind, window, kKeyTile, c_lo, c_hi);
+    row_allowed_cols(Lk, row + q_shift, jt, mask_kind, window, kKeyTile, c_lo, c_hi);
     float s[kKeyTile];
     float mt = -INFINITY;
 #pragma unroll
@@ -142,7 +144,7 @@ int launch_f32_t(const FwdArgs& a, cudaStream_t stream, cudaError_t* err) {
   kernel<<<grid, kThreadsF32, smem, stream>>>(
       static_cast<const float*>(a.q), static_cast<const float*>(a.k),
       static_cast<const float*>(a.v), static_cast<float*>(a.out), a.lse, a.L, a.d, a.scale,
-      a.mask_kind, a.window);
+      a.mask_kind, a.window, a.Lk > 0 ? a.Lk : a.L, a.q_shift);
   *err = cudaGetLastError();
   return *err == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

@@ -142,7 +142,9 @@ struct Cfg {
 struct Params {
   void* out;
   float* lse;
-  int BH, L;
+  int BH, L;      // L query rows per head (q, out, lse)
+  int Lk;         // key rows per head (k, v)
+  int q_shift;    // query row i sits at key position q_shift + i
   int mask_kind, window;
   float scale_log2;  // scale * log2(e)
   int num_units, nqp;
@@ -186,7 +188,8 @@ __device__ __forceinline__ TileWork decode_tile(int u, int t, const Params& p) {
   w.q_last = min(w.q_first + kBM - 1, p.L - 1);
   w.lo = w.hi = 0;
   if (w.valid) {
-    kv_tile_range(p.L, w.q_first, w.q_last, p.mask_kind, p.window, BN, w.lo, w.hi);
+    kv_tile_range(p.Lk, w.q_first + p.q_shift, w.q_last + p.q_shift, p.mask_kind, p.window, BN,
+                  w.lo, w.hi);
     if (p.num_splits > 1) {
       w.lo = max(w.lo, w.split * p.split_blocks);
       w.hi = min(w.hi, (w.split + 1) * p.split_blocks);
@@ -732,7 +735,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!w.valid) continue;
       const int row_a = w.q_first + ra, row_b = w.q_first + rb;
       int full_lo, full_hi;  // key blocks that need no element mask
-      kv_full_range(p.L, w.q_first, w.q_last, p.mask_kind, p.window, BN, full_lo, full_hi);
+      kv_full_range(p.Lk, w.q_first + p.q_shift, w.q_last + p.q_shift, p.mask_kind, p.window, BN,
+                    full_lo, full_hi);
       // per row: running max (log2 units), sum of the probabilities against
       // it and sum of their bf16 roundings
       float m_a = -INFINITY, m_b = -INFINITY;
@@ -768,8 +772,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool full = j >= full_lo && j < full_hi;
         int a_lo = 0, a_hi = BN, b_lo = 0, b_hi = BN;
         if (!full) {
-          row_allowed_cols(p.L, row_a, j, p.mask_kind, p.window, BN, a_lo, a_hi);
-          row_allowed_cols(p.L, row_b, j, p.mask_kind, p.window, BN, b_lo, b_hi);
+          row_allowed_cols(p.Lk, row_a + p.q_shift, j, p.mask_kind, p.window, BN, a_lo, a_hi);
+          row_allowed_cols(p.Lk, row_b + p.q_shift, j, p.mask_kind, p.window, BN, b_lo, b_hi);
           mask_groups<0, kHalf>(s, t0, a_lo, a_hi, b_lo, b_hi);
         }
         EBH_TRACE(kEvMasked, j);
@@ -1081,14 +1085,17 @@ int launch_t(const FwdArgs& a, cudaStream_t stream, cudaError_t* err) {
   const int BH = a.B * a.H;
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, a.q, BH, a.L, D, kBM, err)) return ATTN_ERR_CUDA;
-  if (!make_map(&tk, a.k, BH, a.L, D, BN, err)) return ATTN_ERR_CUDA;
-  if (!make_map(&tv, a.v, BH, a.L, D, BN, err)) return ATTN_ERR_CUDA;
+  const int Lk = a.Lk > 0 ? a.Lk : a.L;
+  if (!make_map(&tk, a.k, BH, Lk, D, BN, err)) return ATTN_ERR_CUDA;
+  if (!make_map(&tv, a.v, BH, Lk, D, BN, err)) return ATTN_ERR_CUDA;
 
   Params p;
   p.out = a.out;
   p.lse = a.lse;
   p.BH = BH;
   p.L = a.L;
+  p.Lk = Lk;
+  p.q_shift = a.q_shift;
   p.mask_kind = a.mask_kind;
   p.window = a.window;
   p.scale_log2 = a.scale * 1.4426950408889634f;

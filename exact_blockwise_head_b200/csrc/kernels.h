@@ -20,6 +20,10 @@ struct FwdArgs {
   int window;       // already clamped to [0, L]
   int block_n;      // 64 or 128 on the bf16 path
   uint64_t timeout_ns;
+  // Query rows at an offset into the keys: q/out/lse have L rows, k/v have Lk
+  // rows (0: Lk = L), and query row i sits at key position q_shift + i.
+  int Lk = 0;
+  int q_shift = 0;
   // split-KV partial mode (bf16 path): when o_part is set, the keys are cut
   // into num_splits runs of split_keys (a multiple of block_n) and the kernel
   // writes fp32 partial O [S,B,H,L,d] and partial LSE [S,B,H,L] instead of
@@ -52,6 +56,10 @@ int launch_fwd_f32(const FwdArgs& a, cudaStream_t stream, cudaError_t* err);
 int launch_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream, cudaError_t* err);
 int launch_merge(const MergeArgs& m, cudaStream_t stream, cudaError_t* err);
 int read_device_status(int device, int reset, cudaError_t* err);
+
+// [S, BH, Ls, d] rank-major rows -> [BH, S Ls, d] (elem_bytes 2 or 4).
+int launch_unshard(const void* src, void* dst, int S, int BH, int Ls, int d, int elem_bytes,
+                   cudaStream_t stream, cudaError_t* err);
 
 // Records e as this thread's attn_last_cuda_error() (defined in api.cpp).
 void set_last_cuda_error(cudaError_t e);

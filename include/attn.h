@@ -130,6 +130,31 @@ typedef struct attn_params {
 /* attn_fwd / attn_fwd_f32 with every knob exposed. */
 ATTN_API int attn_fwd_ex(const attn_params* p, void* stream);
 
+/*
+ * Forward for a block of query rows placed inside a longer key sequence:
+ * q, out are [B, H, L, d] with L = p->L query rows, k, v are [B, H, kv_len, d],
+ * lse is [B, H, L]; query row i sits at key position q_offset + i, and the
+ * masks compare key positions with that position.  With q_offset = 0 and
+ * kv_len = L this is attn_fwd_ex.  This is the local step of sequence-sharded
+ * attention ("Mosaic multi-GPU sequence-sharded attention", section 2.1): a
+ * rank holding query rows [r Ls, (r+1) Ls) runs it against the gathered keys.
+ * Requires 0 <= q_offset and q_offset + L <= kv_len (every row keeps its own
+ * key, so no row is fully masked); window masks are clamped to kv_len.
+ * Both dtypes; other arguments and errors as attn_fwd_ex.
+ */
+ATTN_API int attn_fwd_rows(const attn_params* p, int kv_len, int q_offset, void* stream);
+
+/*
+ * Layout step of sequence-sharded attention: an all-gather of S sequence
+ * shards of K (or V), each [B, H, Ls, d], leaves them rank-major,
+ * gathered = [S, B, H, Ls, d]; this writes out = [B, H, S Ls, d], where shard
+ * g's row c becomes key g Ls + c ("Mosaic multi-GPU sequence-sharded
+ * attention", section 2.1).  elem_bytes 2 (bf16) or 4 (fp32); both buffers
+ * device memory and disjoint.  Asynchronous on `stream`; allocates nothing.
+ */
+ATTN_API int attn_seq_unshard(const void* gathered, void* out, int S, int B, int H, int Ls, int d,
+                              int elem_bytes, void* stream);
+
 /* Static text for a status code (never NULL). */
 ATTN_API const char* attn_strerror(int status);
 

@@ -1,0 +1,93 @@
+"""Sequence-sharded forward across ranks: the orchestration on CPU gloo ranks.
+
+"Mosaic multi-GPU sequence-sharded attention", section 2.1: rank r holds rows
+[r Ls, (r+1) Ls) of Q, K and V.  These tests run the real gather step (a
+torch.distributed collective, here over gloo) with the other two steps done on
+the CPU: the layout change as an array transpose and the local forward by the
+fp64 oracle on the rank's rows.  The rows every rank returns must be the
+unsharded definition's rows.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from exact_blockwise_head_b200 import seqpar
+
+
+def test_shard_offsets():
+    assert [seqpar.shard_offset(128, r) for r in range(4)] == [0, 128, 256, 384]
+    with pytest.raises(ValueError):
+        seqpar.shard_offset(0, 1)
+
+
+class _CpuOps(seqpar.DeviceOps):
+    """gather as on the GPUs; unshard and the local forward on the CPU."""
+
+    def unshard(self, gathered):
+        S, B, H, Ls, d = gathered.shape
+        return gathered.permute(1, 2, 0, 3, 4).reshape(B, H, S * Ls, d)
+
+    def local(self, q, k_full, v_full, q_offset, scale, mask, window, block_n):
+        import oracle
+
+        B, H, Ls, d = q.shape
+        L = k_full.shape[2]
+        q_full = torch.zeros(B, H, L, d)
+        q_full[:, :, q_offset:q_offset + Ls] = q
+        bh = np.repeat(np.arange(B * H), Ls)
+        rows = np.tile(np.arange(q_offset, q_offset + Ls), B * H)
+        o, l = oracle.attention_rows(q_full.numpy(), k_full.numpy(), v_full.numpy(), bh, rows,
+                                     scale=scale, mask=mask, window=window)
+        return o.reshape(B, H, Ls, d), l.reshape(B, H, Ls)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, q, k, v, mask, window, result):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    Ls = q.shape[2] // world
+    sl = slice(rank * Ls, (rank + 1) * Ls)
+    o, l = seqpar.forward(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(),
+                          v[:, :, sl].contiguous(), mask=mask, window=window, ops=_CpuOps())
+    result.put((rank, o, l))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,mask,window", [(2, "causal", 0), (2, "none", 0),
+                                               (2, "window", 9), (3, "causal_window", 13)])
+def test_gloo_ranks_return_their_rows_of_the_definition(world, mask, window):
+    import oracle
+
+    B, H, L, d = 1, 2, 24 * world, 8
+    g = torch.Generator().manual_seed(world * 10 + len(mask))
+    q, k, v = (torch.randn(B, H, L, d, generator=g) for _ in range(3))
+    ctx = mp.get_context("spawn")
+    result = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q, k, v, mask, window, result))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted((result.get(timeout=180) for _ in range(world)), key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    full_o, full_l = oracle.attention(q.numpy(), k.numpy(), v.numpy(), mask=mask, window=window)
+    o = np.concatenate([x[1] for x in got], axis=2)
+    l = np.concatenate([x[2] for x in got], axis=2)
+    assert np.abs(o - full_o).max() <= 1e-12
+    assert np.abs(l - full_l).max() <= 1e-12
