@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference] [--no-sweep] [--cpu-seconds S]
+                    [--parallel heads|seq]
 
 Default workload: the blockwise causal problem B=1, H=32, L=8192, d=128
 (bf16, inputs N(0,1)/sqrt(2)), the configuration the target is stated on.
@@ -74,6 +75,21 @@ def allowed_pairs(L: int, mask: str, window: int) -> int:
     # row i sees keys [max(0, i-w), min(L-1, i+w)]
     total = L * (2 * w + 1)
     total -= w * (w + 1)  # clipped at the left edge (rows 0..w-1) and the right edge
+    return total
+
+
+def allowed_pairs_rows(L: int, a: int, b: int, mask: str, window: int) -> int:
+    """Allowed (i, j) pairs of query rows [a, b) in one head of length L."""
+    total = 0
+    for i in range(a, b):
+        lo, hi = 0, L - 1
+        if mask == "causal":
+            hi = i
+        elif mask == "window":
+            lo, hi = max(0, i - window), min(L - 1, i + window)
+        elif mask == "causal_window":
+            lo, hi = max(0, i - window), i
+        total += hi - lo + 1
     return total
 
 
@@ -273,6 +289,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--parallel", default="heads", choices=["heads", "seq"],
+                    help="heads: shard (batch, head) pairs, no collective (default); "
+                         "seq: shard the sequence, all-gather K/V")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -289,6 +308,8 @@ def main():
 
     if args.impl == "reference":
         return reference_arm(args, w, world, rank)
+    if args.parallel == "seq":
+        return seq_parallel_arm(args, w, world, rank, local_rank)
 
     import torch
     import torch.distributed as dist
@@ -421,6 +442,121 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def seq_parallel_arm(args, w, world, rank, local_rank):
+    """--parallel seq: the workload's sequence is cut into `world` contiguous
+    shards (strong scaling).  A step is seqpar.forward on this rank's shard:
+    all-gather K and V, reorder them, run the rank's query rows."""
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    import exact_blockwise_head_b200 as ebh
+    from exact_blockwise_head_b200 import seqpar
+
+    if w.L % world:
+        raise SystemExit("--parallel seq needs L divisible by the number of GPUs")
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        s = socket.socket()
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+        s.close()
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                world_size=1, timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    Ls = w.L // world
+    a, b = rank * Ls, (rank + 1) * Ls
+    q, k, v = ebh.make_qkv(w)
+    qh, kh, vh = (x[:, :, a:b].contiguous().pin_memory() for x in (q, k, v))
+    del q, k, v
+    qd, kd, vd = (x.cuda() for x in (qh, kh, vh))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        return seqpar.forward(qd, kd, vd, mask=w.mask, window=w.window, block_n=args.block_n)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    with ClockSampler(local_rank) as clk:
+        ms = time_gpu(step, args.steps, stream)
+    dist.barrier()
+    assert ebh.device_status(local_rank) == ebh.ATTN_OK, "a kernel wait ran out"
+    t = torch.tensor([sum(ms)], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_per_step = float(t.item()) / args.steps
+    flops_total = algorithmic_flops(w)
+    value = flops_total / (ms_per_step * 1e-3) / 1e12
+    rank_flops = 4.0 * w.d * w.B * w.H * allowed_pairs_rows(w.L, a, b, w.mask, w.window)
+    own_ms = sum(ms) / len(ms)
+
+    oh = torch.empty(qh.shape, dtype=qh.dtype).pin_memory()
+    lh = torch.empty((w.B, w.H, Ls), dtype=torch.float32).pin_memory()
+    qe, ke, ve = (torch.empty_like(qd) for _ in range(3))
+
+    def e2e_step():
+        qe.copy_(qh, non_blocking=True)
+        ke.copy_(kh, non_blocking=True)
+        ve.copy_(vh, non_blocking=True)
+        o, l = seqpar.forward(qe, ke, ve, mask=w.mask, window=w.window, block_n=args.block_n)
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(l, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, 20))
+    e2e_ms = time_gpu(e2e_step, e2e_steps, stream)
+    e2e_t = torch.tensor([sum(e2e_ms) / e2e_steps], device="cuda", dtype=torch.float64)
+    dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = rank_flops / (own_ms * 1e-3) / 1e12
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "tokens_per_s": round(w.B * w.L / (ms_per_step * 1e-3), 1),
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "strong",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
+                   "mask": w.mask, "window": w.window, "block_n": args.block_n or 128,
+                   "rows_per_gpu": Ls,
+                   "parallelism": f"sequence sharded x{world} (all-gather K/V, then rows)",
+                   "l2": "inputs larger than L2 (126 MB)" if 3 * qd.numel() * 2 * world > 126e6
+                   else "not flushed"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)"
+                     if peak_kind == "measured" else "fallback 1.59 PFLOP/s",
+                     "note": "rank 0's algorithmic FLOPs over its whole step "
+                             "(gather + reorder + forward)",
+                     "traffic": None},
+        "e2e": {"value": round(flops_total / (float(e2e_t.item()) * 1e-3) / 1e12, 2),
+                "unit": "TFLOP/s", "h2d_bytes_per_step": 3 * qd.numel() * 2,
+                "d2h_bytes_per_step": oh.numel() * 2 + lh.numel() * 4},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
 
 
 def reference_arm(args, w, world, rank):

@@ -30,6 +30,15 @@ def test_workload_flop_counts():
     assert abs(bench.algorithmic_flops(w) - 549.8e9) / 549.8e9 < 1e-3
 
 
+@pytest.mark.parametrize("mask,window", [("none", 0), ("causal", 0), ("window", 5),
+                                         ("causal_window", 6)])
+def test_row_range_pairs_add_up(mask, window):
+    L = 48
+    M = np.array(dense_mask(L, mask, window))
+    for a, b in ((0, 48), (0, 12), (12, 30), (30, 48), (47, 48)):
+        assert bench.allowed_pairs_rows(L, a, b, mask, window) == int(M[a:b].sum())
+
+
 @pytest.mark.parametrize("total,world", [(0, 1), (1, 1), (7, 2), (32, 8), (5, 8), (100, 3)])
 def test_shard_range_partitions(total, world):
     seen = []
