@@ -58,8 +58,10 @@ def _bind(path):
                                        ctypes.c_double, ctypes.c_int, i64, i64]
     lib.oracle_attn_partial.argtypes = [f32p, f32p, f32p, f64p, f64p, i64, i64, i64, i64,
                                         ctypes.c_double, ctypes.c_int, i64, i64, i64]
+    lib.oracle_mha_fwd.argtypes = [f32p, f32p, f32p, f32p, f32p, f64p, i64, i64, i64, i64,
+                                   ctypes.c_int, i64]
     for name in ("oracle_attn_fwd", "oracle_attn_rows", "oracle_attn_kv_blockwise",
-                 "oracle_attn_q_blockwise", "oracle_attn_partial"):
+                 "oracle_attn_q_blockwise", "oracle_attn_partial", "oracle_mha_fwd"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -176,6 +178,28 @@ class Oracle:
         return out, lse
 
 
+    def mha(self, x, w_qkv, b_qkv, w_out, b_out, num_heads, mask="none", window=0):
+        """The multi-head attention layer (single thread): x [B, L, E], weights in
+        nn.Linear layout, biases or None; returns y [B, L, E] float64."""
+        def f32(a):
+            return None if a is None else np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+        x, w_qkv, w_out, b_qkv, b_out = (f32(a) for a in (x, w_qkv, w_out, b_qkv, b_out))
+        B, L, E = x.shape
+        if w_qkv.shape != (3 * E, E) or w_out.shape != (E, E):
+            raise ValueError("weights must be [3E, E] and [E, E]")
+        y = np.empty((B, L, E), np.float64)
+        rc = self._lib.oracle_mha_fwd(
+            _ptr(x, ctypes.c_float), _ptr(w_qkv, ctypes.c_float),
+            None if b_qkv is None else _ptr(b_qkv, ctypes.c_float),
+            _ptr(w_out, ctypes.c_float),
+            None if b_out is None else _ptr(b_out, ctypes.c_float),
+            _ptr(y, ctypes.c_double), B, L, E, int(num_heads), MASKS[mask], int(window))
+        if rc != 0:
+            raise RuntimeError(f"oracle_mha_fwd failed ({rc})")
+        return y
+
+
 def load_variant(path: str) -> Oracle:
     """Bind an Oracle to another compiled copy of the source (used by the tests
     that plant a mistake in a copy of the oracle and check that a pin fails)."""
@@ -204,3 +228,7 @@ def attention_q_blockwise(*a, **kw):
 
 def attention_partial(*a, **kw):
     return _default().attention_partial(*a, **kw)
+
+
+def mha(*a, **kw):
+    return _default().mha(*a, **kw)

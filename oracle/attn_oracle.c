@@ -369,3 +369,76 @@ int oracle_attn_partial(const float* q, const float* k, const float* v, double* 
   }
   return 0;
 }
+
+/* ---- the multi-head attention layer [MHA-CUDA 2.1, 2.2] -------------- */
+
+/*
+ * The layer's steps in the page's order, all in fp64:
+ *   qkv = x W_qkv^T + b_qkv                       (Linear(E, 3E))
+ *   q, k, v = qkv[..., 0:E], [E:2E], [2E:3E]      (chunk(3, dim=-1))
+ *   head h of each = columns [h d, (h+1) d)       (view(B, L, H, d).transpose)
+ *   context[b, i, h d + c] = definition row i of head h, scale 1/sqrt(d)
+ *   y = context W_out^T + b_out                   (Linear(E, E))
+ * Biases may be NULL (zero).  Single-threaded; for small problems.
+ */
+int oracle_mha_fwd(const float* x, const float* w_qkv, const float* b_qkv, const float* w_out,
+                   const float* b_out, double* y, int64_t B, int64_t L, int64_t E, int64_t H,
+                   int mask_kind, int64_t window) {
+  if (!x || !w_qkv || !w_out || !y || B <= 0 || L <= 0 || E <= 0 || H <= 0 || E % H) return -1;
+  if (mask_kind < ORACLE_MASK_NONE || mask_kind > ORACLE_MASK_CAUSAL_WINDOW) return -1;
+  if ((mask_kind == ORACLE_MASK_WINDOW || mask_kind == ORACLE_MASK_CAUSAL_WINDOW) && window < 0)
+    return -1;
+  const int64_t d = E / H;
+  const double scale = 1.0 / sqrt((double)d);
+  double* qkv = (double*)malloc((size_t)(B * L * 3 * E) * sizeof(double));
+  double* ctx = (double*)malloc((size_t)(B * L * E) * sizeof(double));
+  double* s = (double*)malloc((size_t)L * sizeof(double));
+  if (!qkv || !ctx || !s) {
+    free(qkv);
+    free(ctx);
+    free(s);
+    return -2;
+  }
+  for (int64_t r = 0; r < B * L; ++r)
+    for (int64_t j = 0; j < 3 * E; ++j) {
+      double acc = b_qkv ? (double)b_qkv[j] : 0.0;
+      for (int64_t c = 0; c < E; ++c) acc += (double)x[r * E + c] * (double)w_qkv[j * E + c];
+      qkv[r * 3 * E + j] = acc;
+    }
+  for (int64_t b = 0; b < B; ++b)
+    for (int64_t h = 0; h < H; ++h)
+      for (int64_t i = 0; i < L; ++i) {
+        const double* qi = qkv + (b * L + i) * 3 * E + h * d;
+        double m = -INFINITY;
+        for (int64_t j = 0; j < L; ++j) {
+          if (!allowed(i, j, mask_kind, window)) continue;
+          const double* kj = qkv + (b * L + j) * 3 * E + E + h * d;
+          double dot = 0.0;
+          for (int64_t c = 0; c < d; ++c) dot += qi[c] * kj[c];
+          s[j] = scale * dot;
+          if (s[j] > m) m = s[j];
+        }
+        double* o = ctx + (b * L + i) * E + h * d;
+        for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+        double l = 0.0;
+        for (int64_t j = 0; j < L; ++j) {
+          if (!allowed(i, j, mask_kind, window)) continue;
+          const double p = exp(s[j] - m);
+          l += p;
+          const double* vj = qkv + (b * L + j) * 3 * E + 2 * E + h * d;
+          for (int64_t c = 0; c < d; ++c) o[c] += p * vj[c];
+        }
+        for (int64_t c = 0; c < d; ++c) o[c] /= l;
+      }
+  for (int64_t r = 0; r < B * L; ++r)
+    for (int64_t j = 0; j < E; ++j) {
+      double acc = b_out ? (double)b_out[j] : 0.0;
+      for (int64_t c = 0; c < E; ++c) acc += ctx[r * E + c] * (double)w_out[j * E + c];
+      y[r * E + j] = acc;
+    }
+  free(qkv);
+  free(ctx);
+  free(s);
+  return 0;
+}
+

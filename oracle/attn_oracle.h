@@ -86,6 +86,13 @@ int oracle_attn_partial(const float* q, const float* k, const float* v, double* 
                         double scale, int mask_kind, int64_t window, int64_t key_lo,
                         int64_t key_hi);
 
+/* The multi-head attention layer of [MHA-CUDA] sections 2.1-2.2: x [B, L, E],
+ * w_qkv [3E, E] and w_out [E, E] in nn.Linear layout, b_qkv [3E] and b_out [E]
+ * (NULL: zero), H heads of d = E / H; y [B, L, E] double. */
+int oracle_mha_fwd(const float* x, const float* w_qkv, const float* b_qkv, const float* w_out,
+                   const float* b_out, double* y, int64_t B, int64_t L, int64_t E, int64_t H,
+                   int mask_kind, int64_t window);
+
 #ifdef __cplusplus
 }
 #endif

@@ -348,3 +348,76 @@ def pin_partials_merge_to_definition(orc):
 ALL_PINS = [pin_brute_force, pin_golden, pin_kv_blockwise, pin_q_blockwise,
             pin_probability_rows, pin_identical_keys, pin_constant_v, pin_special_cases,
             pin_overflow, pin_rows_match, pin_partials_merge_to_definition]
+
+
+# --------------------------------------------------------------------------
+# the multi-head attention layer [MHA-CUDA 2.1, 2.2]
+# --------------------------------------------------------------------------
+def brute_force_mha(x, w_qkv, b_qkv, w_out, b_out, H, mask, window):
+    """The page's layer with plain Python loops, one step per line of its
+    forward: Linear(E, 3E), chunk into q, k, v, split heads, masked softmax
+    attention with 1/sqrt(d), merge heads, Linear(E, E)."""
+    B, L, E = len(x), len(x[0]), len(x[0][0])
+    d = E // H
+    M = dense_mask(L, mask, window)
+
+    def linear(rows, W, b):
+        return [[math.fsum([rows[r][c] * W[j][c] for c in range(len(rows[0]))])
+                 + (b[j] if b is not None else 0.0) for j in range(len(W))]
+                for r in range(len(rows))]
+
+    y = []
+    for bb in range(B):
+        qkv = linear(x[bb], w_qkv, b_qkv)
+        q = [row[0:E] for row in qkv]
+        k = [row[E:2 * E] for row in qkv]
+        v = [row[2 * E:3 * E] for row in qkv]
+        ctx = [[0.0] * E for _ in range(L)]
+        for h in range(H):
+            cols = range(h * d, (h + 1) * d)
+            for i in range(L):
+                e = [math.exp(math.fsum([q[i][c] * k[j][c] for c in cols]) / math.sqrt(d))
+                     if M[i][j] else 0.0 for j in range(L)]
+                Z = math.fsum(e)
+                for c in cols:
+                    ctx[i][c] = math.fsum([e[j] * v[j][c] for j in range(L)]) / Z
+        y.append(linear(ctx, w_out, b_out))
+    return y
+
+
+def pin_mha_brute_force(orc):
+    """The layer against the pure-Python restatement of the page's forward."""
+    rng = np.random.default_rng(40)
+    for (B, L, E, H), (mask, window) in (((1, 4, 4, 2), ("none", 0)), ((2, 5, 6, 3), ("causal", 0)),
+                                         ((1, 6, 4, 1), ("window", 1)),
+                                         ((1, 5, 8, 2), ("causal_window", 2))):
+        x = rng.standard_normal((B, L, E)).astype(np.float32)
+        w_qkv = (rng.standard_normal((3 * E, E)) * 0.5).astype(np.float32)
+        b_qkv = rng.standard_normal(3 * E).astype(np.float32)
+        w_out = (rng.standard_normal((E, E)) * 0.5).astype(np.float32)
+        b_out = rng.standard_normal(E).astype(np.float32)
+        y = orc.mha(x, w_qkv, b_qkv, w_out, b_out, H, mask=mask, window=window)
+        ref = brute_force_mha(x.tolist(), w_qkv.tolist(), b_qkv.tolist(), w_out.tolist(),
+                              b_out.tolist(), H, mask, window)
+        _close(y, ref, 1e-12, 1e-12, f"mha brute force {B, L, E, H} {mask}")
+        y0 = orc.mha(x, w_qkv, None, w_out, None, H, mask=mask, window=window)
+        ref0 = brute_force_mha(x.tolist(), w_qkv.tolist(), None, w_out.tolist(), None, H, mask,
+                               window)
+        _close(y0, ref0, 1e-12, 1e-12, f"mha brute force, no biases {mask}")
+
+
+def pin_mha_identity_projections(orc):
+    """With W_qkv = [I; I; I], W_out = I and zero biases the layer is the
+    attention of x split into heads, merged back (checked against the pinned
+    attention functions)."""
+    B, L, E, H = 2, 30, 12, 3
+    d = E // H
+    x = _rand((B, L, E), 41)
+    eye = np.eye(E, dtype=np.float32)
+    y = orc.mha(x, np.concatenate([eye, eye, eye]), None, eye, None, H, mask="causal")
+    heads = x.reshape(B, L, H, d).transpose(0, 2, 1, 3).copy()
+    o, _ = orc.attention(heads, heads, heads, scale=1.0 / math.sqrt(d), mask="causal")
+    _close(y, o.transpose(0, 2, 1, 3).reshape(B, L, E), 1e-13, 1e-13, "identity projections")
+
+
+ALL_PINS += [pin_mha_brute_force, pin_mha_identity_projections]

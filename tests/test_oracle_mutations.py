@@ -35,6 +35,11 @@ MUTANTS = [
      "int64_t i1 = i0 + block < L ? i0 + block : L - 1;"),
     ("causal_window_two_sided", "(j <= i) && (i - j <= window)", "(i - j <= window)"),
     ("causal_window_off_by_one", "(j <= i) && (i - j <= window)", "(j <= i) && (i - j < window)"),
+    ("mha_out_bias_dropped", "double acc = b_out ? (double)b_out[j] : 0.0;", "double acc = 0.0;"),
+    ("mha_k_read_from_q_block", "qkv + (b * L + j) * 3 * E + E + h * d;",
+     "qkv + (b * L + j) * 3 * E + h * d;"),
+    ("mha_head_offset_wrong", "const double* qi = qkv + (b * L + i) * 3 * E + h * d;",
+     "const double* qi = qkv + (b * L + i) * 3 * E + h;"),
     ("partial_not_normalised", "for (int64_t c = 0; c < d; ++c) o[c] /= l;\n      lse[bh * L + i]",
      "lse[bh * L + i]"),
     ("partial_range_shifted", "for (int64_t j = key_lo; j < key_hi; ++j) {\n        if (!allowed(i, j, mask_kind, window)) continue;\n        double dot = 0.0;\n        for (int64_t c = 0; c < d; ++c) dot += (double)qi[c] * (double)kh[j * d + c];\n        double p",
