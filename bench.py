@@ -278,6 +278,36 @@ def sweep_other(ebh, torch, names, steps=5, warmup=3):
     return res
 
 
+def sweep_layer(ebh, torch, B=4, L=2048, E=512, H=8, steps=10):
+    """The whole multi-head attention layer of the MHA page (qkv projection,
+    head split, attention, merge, out projection), at the 8-head L=2048,
+    E=512 configuration, L2 flushed between steps."""
+    a = 1.0 / math.sqrt(E)
+    x = torch.randn(B, L, E, device="cuda").to(torch.bfloat16)
+    w_qkv = ((torch.rand(3 * E, E, device="cuda") * 2 - 1) * a).to(torch.bfloat16)
+    b_qkv = ((torch.rand(3 * E, device="cuda") * 2 - 1) * a).to(torch.bfloat16)
+    w_out = ((torch.rand(E, E, device="cuda") * 2 - 1) * a).to(torch.bfloat16)
+    b_out = ((torch.rand(E, device="cuda") * 2 - 1) * a).to(torch.bfloat16)
+    y = torch.empty_like(x)
+    ws = torch.empty(ebh.mha_workspace_bytes(B, L, E) + 256, dtype=torch.uint8, device="cuda")
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def fn():
+        ebh.mha_forward(x, w_qkv, b_qkv, w_out, b_out, H, y=y, workspace=ws)
+
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    ms = time_gpu(fn, steps, torch.cuda.current_stream(), flush=lambda: flush_buf.zero_())
+    avg = sum(ms) / len(ms)
+    flops = 8.0 * B * L * E * E + 4.0 * B * H * L * L * (E // H)
+    return {"ms": round(avg, 4), "tokens_per_s": round(B * L / avg * 1e3, 1),
+            "tflops": round(flops / avg / 1e9, 1),
+            "config": f"B={B} L={L} E={E} H={H}, no mask, bf16",
+            "l2": "flushed between steps",
+            "flops": "8 B L E^2 (projections) + 4 B H L^2 d (attention)"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,6 +465,7 @@ def main():
                   if n != w.name]
         del qe, ke, ve
         line["other_workloads_kernel_only"] = sweep_other(ebh, torch, others)
+        line["mha_layer"] = sweep_layer(ebh, torch)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, q, k, v, args.cpu_seconds)
     if world > 1:

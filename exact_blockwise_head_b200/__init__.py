@@ -38,7 +38,7 @@ EXPORTED = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ex", "attn_strerror", "attn_la
             "attn_device_status", "attn_selftest_wait_timeout", "attn_kv_tile_range",
             "attn_kv_tile_class", "attn_kv_full_range", "attn_splitkv_workspace_bytes",
             "attn_fwd_splitkv", "attn_merge", "attn_abi_version", "attn_fwd_splitkv_noalloc",
-            "attn_fwd_rows", "attn_seq_unshard")
+            "attn_fwd_rows", "attn_seq_unshard", "attn_mha_workspace_bytes", "attn_mha_fwd")
 
 
 class AttnParams(ctypes.Structure):
@@ -59,6 +59,24 @@ class AttnParams(ctypes.Structure):
         ("window", ctypes.c_int),
         ("block_n", ctypes.c_int),
         ("wait_timeout_ns", ctypes.c_uint64),
+    ]
+
+
+class MhaParams(ctypes.Structure):
+    """Mirror of ``attn_mha_params`` in include/attn.h."""
+    _fields_ = [
+        ("x", ctypes.c_void_p),
+        ("w_qkv", ctypes.c_void_p),
+        ("b_qkv", ctypes.c_void_p),
+        ("w_out", ctypes.c_void_p),
+        ("b_out", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+        ("B", ctypes.c_int),
+        ("L", ctypes.c_int),
+        ("E", ctypes.c_int),
+        ("H", ctypes.c_int),
+        ("mask_kind", ctypes.c_int),
+        ("window", ctypes.c_int),
     ]
 
 
@@ -105,12 +123,15 @@ def _load():
             lib.attn_fwd_splitkv_noalloc.argtypes = [ctypes.POINTER(AttnParams), i, vp]
             lib.attn_fwd_rows.argtypes = [ctypes.POINTER(AttnParams), i, i, vp]
             lib.attn_seq_unshard.argtypes = [vp, vp, i, i, i, i, i, i, vp]
+            lib.attn_mha_workspace_bytes.argtypes = [i, i, i]
+            lib.attn_mha_fwd.argtypes = [ctypes.POINTER(MhaParams), vp, ctypes.c_size_t, vp]
             lib.attn_merge.argtypes = [vp, vp, i, ctypes.POINTER(i), i, i, vp, vp, i, i, i, i, i,
                                        vp]
             for name in EXPORTED:
                 if name != "attn_strerror":
                     getattr(lib, name).restype = ctypes.c_int
             lib.attn_splitkv_workspace_bytes.restype = ctypes.c_size_t
+            lib.attn_mha_workspace_bytes.restype = ctypes.c_size_t
             _lib = lib
     return _lib
 
@@ -238,6 +259,53 @@ def seq_unshard(gathered, out=None, stream=None):
     if st != ATTN_OK:
         raise AttnError(st, "attn_seq_unshard")
     return out
+
+
+def mha_workspace_bytes(B, L, E) -> int:
+    return int(_load().attn_mha_workspace_bytes(B, L, E))
+
+
+def mha_forward(x, w_qkv, b_qkv, w_out, b_out, num_heads, mask="none", window=0, y=None,
+                workspace=None, stream=None):
+    """The multi-head attention layer: y = out_proj(attention(split(qkv_proj(x)))).
+    x: bf16 [B, L, E]; w_qkv [3E, E], b_qkv [3E] (or None), w_out [E, E],
+    b_out [E] (or None), all bf16 CUDA tensors in nn.Linear layout; E /
+    num_heads in {64, 128}.  `workspace` is a CUDA uint8 tensor of at least
+    mha_workspace_bytes(B, L, E) bytes (allocated here when omitted)."""
+    import torch
+
+    if x.dim() != 3 or x.dtype != torch.bfloat16:
+        raise ValueError("x must be a bf16 [B, L, E] tensor")
+    B, L, E = x.shape
+    for name, t, shape in (("w_qkv", w_qkv, (3 * E, E)), ("w_out", w_out, (E, E)),
+                           ("b_qkv", b_qkv, (3 * E,)), ("b_out", b_out, (E,))):
+        if t is None and name.startswith("b_"):
+            continue
+        if tuple(t.shape) != shape or t.dtype != torch.bfloat16 or not t.is_cuda or \
+                not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor of shape {shape}")
+    if mask not in MASK_KINDS:
+        raise ValueError(f"mask must be one of {sorted(MASK_KINDS)}")
+    if y is None:
+        y = torch.empty_like(x)
+    need = mha_workspace_bytes(B, L, E)
+    if workspace is None:
+        workspace = torch.empty(need + 256, dtype=torch.uint8, device=x.device)
+    base = workspace.data_ptr()
+    pad = (-base) % 256
+    p = MhaParams()
+    p.x, p.w_qkv, p.w_out, p.y = x.data_ptr(), w_qkv.data_ptr(), w_out.data_ptr(), y.data_ptr()
+    p.b_qkv = b_qkv.data_ptr() if b_qkv is not None else None
+    p.b_out = b_out.data_ptr() if b_out is not None else None
+    p.B, p.L, p.E, p.H = B, L, E, int(num_heads)
+    p.mask_kind = MASK_KINDS[mask]
+    p.window = int(window)
+    with torch.cuda.device(x.device):
+        st = _load().attn_mha_fwd(ctypes.byref(p), ctypes.c_void_p(base + pad),
+                                  workspace.numel() - pad, _stream_handle(stream, x.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_mha_fwd")
+    return y
 
 
 def _params(q, k, v, scale, mask, window, block_n, out, lse, want_lse, wait_timeout_ns):

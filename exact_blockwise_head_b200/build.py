@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libebh_attn.so")
 TRACE_LIB = os.path.join(PKG, "libebh_attn_trace.so")
 SOURCES = ["api.cpp", "attn_sm100.cu", "attn_f32.cu", "attn_merge.cu", "noalloc.cu",
-           "seqpar.cu"]
+           "seqpar.cu", "mha.cu"]
 HEADERS = ["kernels.h", "sm100_ptx.cuh", "tiles.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -68,6 +68,7 @@ def build(force: bool = False, verbose: bool = False, trace: bool = False,
     if verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
+    cmd += ["-lcublasLt"]  # the layer's two projections
     subprocess.run(cmd, check=True)
     os.replace(tmp, target)
     return target

@@ -184,6 +184,65 @@ int attn_seq_unshard(const void* gathered, void* out, int S, int B, int H, int L
   return st;
 }
 
+size_t attn_mha_workspace_bytes(int B, int L, int E) {
+  if (B <= 0 || L <= 0 || E <= 0) return 0;
+  return ebh::mha_workspace_bytes(B, L, E);
+}
+
+int attn_mha_fwd(const attn_mha_params* p, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  if (p == nullptr || !p->x || !p->w_qkv || !p->w_out || !p->y || !workspace)
+    return ATTN_ERR_INVALID;
+  if (p->B <= 0 || p->L <= 0 || p->E <= 0 || p->H <= 0 || p->E % p->H != 0)
+    return ATTN_ERR_INVALID;
+  if (static_cast<long long>(p->B) * p->H > 0x7fffffffLL ||
+      static_cast<long long>(p->B) * p->L > 0x7fffffffLL)
+    return ATTN_ERR_INVALID;
+  if (p->mask_kind < ATTN_MASK_NONE || p->mask_kind > ATTN_MASK_CAUSAL_WINDOW) return ATTN_ERR_INVALID;
+  if (has_window(p->mask_kind) && p->window < 0) return ATTN_ERR_INVALID;
+  const int d = p->E / p->H;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  const size_t need = ebh::mha_workspace_bytes(p->B, p->L, p->E);
+  if (workspace_bytes < need) return ATTN_ERR_INVALID;
+  if (!aligned(workspace, 256)) return ATTN_ERR_MISALIGNED;
+  if (!aligned(p->x, 16) || !aligned(p->w_qkv, 16) || !aligned(p->w_out, 16) ||
+      !aligned(p->y, 16) || (p->b_qkv && !aligned(p->b_qkv, 16)) ||
+      (p->b_out && !aligned(p->b_out, 16)))
+    return ATTN_ERR_MISALIGNED;
+  {
+    const uint64_t act = static_cast<uint64_t>(p->B) * p->L * p->E * 2;
+    const uint64_t wq = static_cast<uint64_t>(3) * p->E * p->E * 2;
+    const uint64_t wo = static_cast<uint64_t>(p->E) * p->E * 2;
+    if (overlap(workspace, need, p->x, act) || overlap(workspace, need, p->y, act) ||
+        overlap(workspace, need, p->w_qkv, wq) || overlap(workspace, need, p->w_out, wo) ||
+        overlap(p->y, act, p->x, act) || overlap(p->y, act, p->w_qkv, wq) ||
+        overlap(p->y, act, p->w_out, wo))
+      return ATTN_ERR_INVALID;
+  }
+  int st = check_device_sm100();
+  if (st != ATTN_OK) return st;
+  ebh::MhaArgs a;
+  a.x = p->x;
+  a.w_qkv = p->w_qkv;
+  a.b_qkv = p->b_qkv;
+  a.w_out = p->w_out;
+  a.b_out = p->b_out;
+  a.y = p->y;
+  a.B = p->B;
+  a.L = p->L;
+  a.E = p->E;
+  a.H = p->H;
+  a.scale = 1.0f / std::sqrt(static_cast<float>(d));
+  a.mask_kind = p->mask_kind;
+  a.window = has_window(p->mask_kind) ? (p->window > p->L ? p->L : p->window) : 0;
+  a.timeout_ns = kDefaultTimeoutNs;
+  cudaError_t err = cudaSuccess;
+  int lt = 0;
+  st = ebh::launch_mha(a, workspace, static_cast<cudaStream_t>(stream), &err, &lt);
+  if (st == ATTN_ERR_CUDA) g_last_cuda_error = lt != 0 ? -lt : static_cast<int>(err);
+  return st;
+}
+
 int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
              int L, int d, float scale, int mask_kind, int window, void* stream) {
   attn_params p = {};

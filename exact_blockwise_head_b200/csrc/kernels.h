@@ -61,6 +61,24 @@ int read_device_status(int device, int reset, cudaError_t* err);
 int launch_unshard(const void* src, void* dst, int S, int BH, int Ls, int d, int elem_bytes,
                    cudaStream_t stream, cudaError_t* err);
 
+// The multi-head attention layer (validated).
+struct MhaArgs {
+  const void* x;       // bf16 [B, L, E]
+  const void* w_qkv;   // bf16 [3E, E]
+  const void* b_qkv;   // bf16 [3E] or nullptr
+  const void* w_out;   // bf16 [E, E]
+  const void* b_out;   // bf16 [E] or nullptr
+  void* y;             // bf16 [B, L, E]
+  int B, L, E, H;
+  float scale;
+  int mask_kind, window;
+  uint64_t timeout_ns;
+};
+size_t mha_workspace_bytes(int B, int L, int E);
+// On ATTN_ERR_CUDA, *err holds a CUDA error or *lt_status a cuBLASLt failure.
+int launch_mha(const MhaArgs& a, void* workspace, cudaStream_t stream, cudaError_t* err,
+               int* lt_status);
+
 // Records e as this thread's attn_last_cuda_error() (defined in api.cpp).
 void set_last_cuda_error(cudaError_t e);
 

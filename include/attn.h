@@ -263,6 +263,39 @@ ATTN_API int attn_merge(const float* o_parts, const float* lse_parts, int num_sp
 #define ATTN_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 ATTN_API int attn_fwd_splitkv_noalloc(const attn_params* p, int num_splits, void* stream);
 
+/*
+ * The multi-head attention layer of "Transformer multi-head attention, 8-head
+ * parallel computation" (lshu.cn), sections 2.1 and 2.2:
+ *   qkv = x W_qkv^T + b_qkv; q, k, v = its three E-wide thirds, each split
+ *   into H heads of d = E / H; context = attention(q, k, v) with scale
+ *   1/sqrt(d) and the mask; y = context W_out^T + b_out.
+ * x, y: bf16 [B, L, E]; w_qkv: bf16 [3E, E] (nn.Linear layout: row j makes
+ * output feature j; rows [0, E) make q, [E, 2E) k, [2E, 3E) v); w_out: bf16
+ * [E, E]; b_qkv [3E] and b_out [E]: bf16 or NULL.  d in {64, 128}; every
+ * pointer 16-byte aligned.  The projections run in cuBLASLt (fp32
+ * accumulation, bias in its epilogue, bf16 results); the head split and merge
+ * and the attention run in this library's kernels.  q, k, v, the attention
+ * output and the context are bf16 in `workspace`: device memory, 256-byte
+ * aligned, at least attn_mha_workspace_bytes(B, L, E) bytes, disjoint from
+ * the other arguments.  On a cuBLASLt failure the call returns ATTN_ERR_CUDA
+ * and attn_last_cuda_error() returns -(1 for the first projection, 2 for the
+ * second).  Asynchronous on `stream`.
+ */
+typedef struct {
+  const void* x;
+  const void* w_qkv;
+  const void* b_qkv;
+  const void* w_out;
+  const void* b_out;
+  void* y;
+  int B, L, E, H;
+  int mask_kind;
+  int window;
+} attn_mha_params;
+ATTN_API size_t attn_mha_workspace_bytes(int B, int L, int E);
+ATTN_API int attn_mha_fwd(const attn_mha_params* p, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
 /* ATTN_ABI_VERSION of the loaded library. */
 ATTN_API int attn_abi_version(void);
 

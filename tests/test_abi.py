@@ -37,6 +37,14 @@ def test_every_declared_symbol_is_exported(lib):
     assert exported == declared_symbols()
 
 
+def test_mha_argument_checks_without_a_device(lib):
+    p = ebh.MhaParams()
+    assert lib.attn_mha_fwd(None, None, 0, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_mha_fwd(ctypes.byref(p), None, 0, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_mha_workspace_bytes(0, 1, 64) == 0
+    assert lib.attn_mha_workspace_bytes(1, 8, 64) > 8 * 64 * 2 * 8
+
+
 def test_abi_version_and_strerror(lib):
     assert lib.attn_abi_version() == 1
     for code in range(0, 6):
