@@ -60,8 +60,11 @@ def _bind(path):
                                         ctypes.c_double, ctypes.c_int, i64, i64, i64]
     lib.oracle_mha_fwd.argtypes = [f32p, f32p, f32p, f32p, f32p, f64p, i64, i64, i64, i64,
                                    ctypes.c_int, i64]
+    lib.oracle_attn_bwd.argtypes = [f32p, f32p, f32p, f32p, f64p, f64p, f64p, i64, i64, i64, i64,
+                                    ctypes.c_double, ctypes.c_int, i64]
     for name in ("oracle_attn_fwd", "oracle_attn_rows", "oracle_attn_kv_blockwise",
-                 "oracle_attn_q_blockwise", "oracle_attn_partial", "oracle_mha_fwd"):
+                 "oracle_attn_q_blockwise", "oracle_attn_partial", "oracle_mha_fwd",
+                 "oracle_attn_bwd"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -200,6 +203,20 @@ class Oracle:
         return y
 
 
+    def attention_backward(self, q, k, v, dout, scale=None, mask="none", window=0):
+        """dQ, dK, dV of the definition given dO (single thread), float64."""
+        q, k, v, B, H, L, d, scale, mk, w = _common(q, k, v, scale, mask, window)
+        g = _f32(dout)
+        dq, dk, dv = (np.empty((B, H, L, d), np.float64) for _ in range(3))
+        rc = self._lib.oracle_attn_bwd(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                       _ptr(v, ctypes.c_float), _ptr(g, ctypes.c_float),
+                                       _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double),
+                                       _ptr(dv, ctypes.c_double), B, H, L, d, scale, mk, w)
+        if rc != 0:
+            raise RuntimeError(f"oracle_attn_bwd failed ({rc})")
+        return dq, dk, dv
+
+
 def load_variant(path: str) -> Oracle:
     """Bind an Oracle to another compiled copy of the source (used by the tests
     that plant a mistake in a copy of the oracle and check that a pin fails)."""
@@ -232,3 +249,7 @@ def attention_partial(*a, **kw):
 
 def mha(*a, **kw):
     return _default().mha(*a, **kw)
+
+
+def attention_backward(*a, **kw):
+    return _default().attention_backward(*a, **kw)

@@ -442,3 +442,75 @@ int oracle_mha_fwd(const float* x, const float* w_qkv, const float* b_qkv, const
   return 0;
 }
 
+/* ---- backward by recomputation [LONGSEQ 3.1], [MOSAIC 2.2] ------------ */
+
+/*
+ * Gradients of O = softmax(scale Q K^T + mask) V given dO, from the
+ * definition (the pages recompute the attention weights instead of storing
+ * them; here every row's weights are recomputed from Q and K):
+ *   P_ij  = exp(s_ij - lse_i) for allowed j, s_ij = scale <q_i, k_j>
+ *   dV_j  = sum_i P_ij dO_i
+ *   dP_ij = <dO_i, v_j>
+ *   D_i   = sum_j P_ij dP_ij
+ *   dS_ij = P_ij (dP_ij - D_i)
+ *   dQ_i  = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i
+ * All [B, H, L, d] in fp64; single-threaded.
+ */
+int oracle_attn_bwd(const float* q, const float* k, const float* v, const float* dout,
+                    double* dq, double* dk, double* dv, int64_t B, int64_t H, int64_t L,
+                    int64_t d, double scale, int mask_kind, int64_t window) {
+  if (check_args(q, k, v, dq, dk, B, H, L, d, mask_kind, window) || !dout || !dv) return -1;
+  double* P = (double*)malloc((size_t)L * sizeof(double));
+  double* dP = (double*)malloc((size_t)L * sizeof(double));
+  if (!P || !dP) {
+    free(P);
+    free(dP);
+    return -2;
+  }
+  const int64_t n = B * H * L * d;
+  for (int64_t e = 0; e < n; ++e) dq[e] = dk[e] = dv[e] = 0.0;
+  for (int64_t bh = 0; bh < B * H; ++bh) {
+    const int64_t head = bh * L * d;
+    for (int64_t i = 0; i < L; ++i) {
+      const float* qi = q + head + i * d;
+      const float* gi = dout + head + i * d;
+      double m = -INFINITY;
+      for (int64_t j = 0; j < L; ++j) {
+        if (!allowed(i, j, mask_kind, window)) continue;
+        double dot = 0.0;
+        for (int64_t c = 0; c < d; ++c) dot += (double)qi[c] * (double)k[head + j * d + c];
+        P[j] = scale * dot;
+        if (P[j] > m) m = P[j];
+      }
+      if (m == -INFINITY) continue; /* no allowed key: no gradient */
+      double l = 0.0;
+      for (int64_t j = 0; j < L; ++j) {
+        if (!allowed(i, j, mask_kind, window)) continue;
+        P[j] = exp(P[j] - m);
+        l += P[j];
+      }
+      double D = 0.0;
+      for (int64_t j = 0; j < L; ++j) {
+        if (!allowed(i, j, mask_kind, window)) continue;
+        P[j] /= l;
+        double dot = 0.0;
+        for (int64_t c = 0; c < d; ++c) dot += (double)gi[c] * (double)v[head + j * d + c];
+        dP[j] = dot;
+        D += P[j] * dot;
+      }
+      for (int64_t j = 0; j < L; ++j) {
+        if (!allowed(i, j, mask_kind, window)) continue;
+        const double ds = P[j] * (dP[j] - D);
+        for (int64_t c = 0; c < d; ++c) {
+          dv[head + j * d + c] += P[j] * (double)gi[c];
+          dq[head + i * d + c] += scale * ds * (double)k[head + j * d + c];
+          dk[head + j * d + c] += scale * ds * (double)qi[c];
+        }
+      }
+    }
+  }
+  free(P);
+  free(dP);
+  return 0;
+}
+

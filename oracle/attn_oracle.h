@@ -93,6 +93,12 @@ int oracle_mha_fwd(const float* x, const float* w_qkv, const float* b_qkv, const
                    const float* b_out, double* y, int64_t B, int64_t L, int64_t E, int64_t H,
                    int mask_kind, int64_t window);
 
+/* Backward by recomputation ([LONGSEQ] 3.1, [MOSAIC] 2.2): dQ, dK, dV of the
+ * definition given dO, all [B, H, L, d] (dq, dk, dv in double). */
+int oracle_attn_bwd(const float* q, const float* k, const float* v, const float* dout,
+                    double* dq, double* dk, double* dv, int64_t B, int64_t H, int64_t L,
+                    int64_t d, double scale, int mask_kind, int64_t window);
+
 #ifdef __cplusplus
 }
 #endif

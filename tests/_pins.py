@@ -421,3 +421,61 @@ def pin_mha_identity_projections(orc):
 
 
 ALL_PINS += [pin_mha_brute_force, pin_mha_identity_projections]
+
+
+# --------------------------------------------------------------------------
+# backward by recomputation [LONGSEQ 3.1], [MOSAIC 2.2]
+# --------------------------------------------------------------------------
+def _grid_values(shape, seed):
+    """Values k / 64, |k| <= 64: x +- 2^-12 is exact in fp32, so central
+    differences see exactly the perturbation they intend."""
+    rng = np.random.default_rng(seed)
+    return (rng.integers(-64, 65, size=shape) / 64.0).astype(np.float32)
+
+
+def pin_backward_finite_differences(orc):
+    """dQ, dK, dV against central differences of the (pinned) forward:
+    f = sum(G * O), df/dx ~ (f(x + e) - f(x - e)) / 2e with e = 2^-12."""
+    B, H, L, d = 1, 1, 5, 3
+    eps = 2.0 ** -12
+    for mask, window in (("none", 0), ("causal", 0), ("window", 1), ("causal_window", 2)):
+        q, k, v, g = (_grid_values((B, H, L, d), s) for s in (50, 51, 52, 53))
+        scale = 0.7
+        dq, dk, dv = orc.attention_backward(q, k, v, g, scale=scale, mask=mask, window=window)
+
+        def f(q_, k_, v_):
+            o, _ = orc.attention(q_, k_, v_, scale=scale, mask=mask, window=window)
+            return math.fsum((o * g.astype(np.float64)).ravel().tolist())
+
+        for name, arr, grad in (("dq", q, dq), ("dk", k, dk), ("dv", v, dv)):
+            num = np.zeros_like(grad)
+            for idx in np.ndindex(arr.shape):
+                up, dn = arr.copy(), arr.copy()
+                up[idx] += eps
+                dn[idx] -= eps
+                args_up = [q, k, v]
+                args_dn = [q, k, v]
+                pos = {"dq": 0, "dk": 1, "dv": 2}[name]
+                args_up[pos], args_dn[pos] = up, dn
+                num[idx] = (f(*args_up) - f(*args_dn)) / (2 * eps)
+            _close(grad, num, 1e-5, 1e-6, f"finite differences {name} {mask}")
+
+
+def pin_backward_invariants(orc):
+    """Constant V: the output ignores Q and K, so dQ = dK = 0.  A common shift
+    of every key leaves each row's softmax unchanged, so sum_j dK_j = 0.
+    Rows of P sum to 1, so sum_j dV_j = sum_i dO_i."""
+    B, H, L, d = 2, 2, 37, 8
+    q, k, g = _rand((B, H, L, d), 54), _rand((B, H, L, d), 55), _rand((B, H, L, d), 56)
+    for mask, window in (("none", 0), ("causal", 0), ("window", 5), ("causal_window", 7)):
+        c = np.broadcast_to(_rand((B, H, 1, d), 57), (B, H, L, d)).copy()
+        dq, dk, _ = orc.attention_backward(q, k, c, g, mask=mask, window=window)
+        assert np.abs(dq).max() <= 1e-13 and np.abs(dk).max() <= 1e-13, mask
+        v = _rand((B, H, L, d), 58)
+        dq, dk, dv = orc.attention_backward(q, k, v, g, mask=mask, window=window)
+        assert np.abs(dk.sum(axis=2)).max() <= 1e-12, mask
+        _close(dv.sum(axis=2), g.astype(np.float64).sum(axis=2), 1e-12, 1e-12,
+               f"sum dV = sum dO {mask}")
+
+
+ALL_PINS += [pin_backward_finite_differences, pin_backward_invariants]

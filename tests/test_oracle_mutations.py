@@ -40,6 +40,11 @@ MUTANTS = [
      "qkv + (b * L + j) * 3 * E + h * d;"),
     ("mha_head_offset_wrong", "const double* qi = qkv + (b * L + i) * 3 * E + h * d;",
      "const double* qi = qkv + (b * L + i) * 3 * E + h;"),
+    ("bwd_D_sign", "const double ds = P[j] * (dP[j] - D);", "const double ds = P[j] * (dP[j] + D);"),
+    ("bwd_dk_missing_scale", "dk[head + j * d + c] += scale * ds * (double)qi[c];",
+     "dk[head + j * d + c] += ds * (double)qi[c];"),
+    ("bwd_dv_at_query_row", "dv[head + j * d + c] += P[j] * (double)gi[c];",
+     "dv[head + i * d + c] += P[j] * (double)gi[c];"),
     ("partial_not_normalised", "for (int64_t c = 0; c < d; ++c) o[c] /= l;\n      lse[bh * L + i]",
      "lse[bh * L + i]"),
     ("partial_range_shifted", "for (int64_t j = key_lo; j < key_hi; ++j) {\n        if (!allowed(i, j, mask_kind, window)) continue;\n        double dot = 0.0;\n        for (int64_t c = 0; c < d; ++c) dot += (double)qi[c] * (double)kh[j * d + c];\n        double p",
