@@ -38,7 +38,8 @@ EXPORTED = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ex", "attn_strerror", "attn_la
             "attn_device_status", "attn_selftest_wait_timeout", "attn_kv_tile_range",
             "attn_kv_tile_class", "attn_kv_full_range", "attn_splitkv_workspace_bytes",
             "attn_fwd_splitkv", "attn_merge", "attn_abi_version", "attn_fwd_splitkv_noalloc",
-            "attn_fwd_rows", "attn_seq_unshard", "attn_mha_workspace_bytes", "attn_mha_fwd")
+            "attn_fwd_rows", "attn_seq_unshard", "attn_mha_workspace_bytes", "attn_mha_fwd",
+            "attn_bwd_workspace_bytes", "attn_bwd", "attn_query_rows_for_keys")
 
 
 class AttnParams(ctypes.Structure):
@@ -124,6 +125,11 @@ def _load():
             lib.attn_fwd_rows.argtypes = [ctypes.POINTER(AttnParams), i, i, vp]
             lib.attn_seq_unshard.argtypes = [vp, vp, i, i, i, i, i, i, vp]
             lib.attn_mha_workspace_bytes.argtypes = [i, i, i]
+            lib.attn_bwd_workspace_bytes.argtypes = [i, i, i]
+            lib.attn_query_rows_for_keys.argtypes = [i, i, i, i, i, ctypes.POINTER(i),
+                                                     ctypes.POINTER(i)]
+            lib.attn_bwd.argtypes = [ctypes.POINTER(AttnParams), vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                     vp]
             lib.attn_mha_fwd.argtypes = [ctypes.POINTER(MhaParams), vp, ctypes.c_size_t, vp]
             lib.attn_merge.argtypes = [vp, vp, i, ctypes.POINTER(i), i, i, vp, vp, i, i, i, i, i,
                                        vp]
@@ -132,6 +138,7 @@ def _load():
                     getattr(lib, name).restype = ctypes.c_int
             lib.attn_splitkv_workspace_bytes.restype = ctypes.c_size_t
             lib.attn_mha_workspace_bytes.restype = ctypes.c_size_t
+            lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
             _lib = lib
     return _lib
 
@@ -259,6 +266,33 @@ def seq_unshard(gathered, out=None, stream=None):
     if st != ATTN_OK:
         raise AttnError(st, "attn_seq_unshard")
     return out
+
+
+def backward(q, k, v, out, lse, dout, scale=None, mask="none", window=0, dq=None, dk=None,
+             dv=None, workspace=None, stream=None):
+    """dQ, dK, dV (fp32) of forward(q, k, v) given dO, recomputing the weights
+    from q, k and the forward's `lse`.  q, k, v, out, dout: one dtype (bf16 or
+    fp32) and one [B, H, L, d] shape; lse: fp32 [B, H, L]."""
+    import torch
+
+    p, _, _ = _params(q, k, v, scale, mask, window, 0, out, lse, True, 0)
+    if dout.shape != q.shape or dout.dtype != q.dtype or not dout.is_cuda or \
+            not dout.is_contiguous():
+        raise ValueError("dout must match q")
+    B, H, L, d = q.shape
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dq is None else dq
+    dk = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dk is None else dk
+    dv = torch.empty(q.shape, dtype=torch.float32, device=q.device) if dv is None else dv
+    need = int(_load().attn_bwd_workspace_bytes(B, H, L))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        st = _load().attn_bwd(ctypes.byref(p), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                              dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                              _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd")
+    return dq, dk, dv
 
 
 def mha_workspace_bytes(B, L, E) -> int:
@@ -434,6 +468,16 @@ def kv_full_range(L, q_first, q_last, mask="none", window=0, block_n=128):
                                     ctypes.byref(lo), ctypes.byref(hi))
     if st != ATTN_OK:
         raise AttnError(st, "attn_kv_full_range")
+    return lo.value, hi.value
+
+
+def query_rows_for_keys(L, k_first, k_last, mask="none", window=0):
+    """Query rows [lo, hi) that may attend to some key in [k_first, k_last]."""
+    lo, hi = ctypes.c_int(), ctypes.c_int()
+    st = _load().attn_query_rows_for_keys(L, k_first, k_last, MASK_KINDS[mask], window,
+                                          ctypes.byref(lo), ctypes.byref(hi))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_query_rows_for_keys")
     return lo.value, hi.value
 
 

@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libebh_attn.so")
 TRACE_LIB = os.path.join(PKG, "libebh_attn_trace.so")
 SOURCES = ["api.cpp", "attn_sm100.cu", "attn_f32.cu", "attn_merge.cu", "noalloc.cu",
-           "seqpar.cu", "mha.cu"]
+           "seqpar.cu", "mha.cu", "attn_bwd.cu"]
 HEADERS = ["kernels.h", "sm100_ptx.cuh", "tiles.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

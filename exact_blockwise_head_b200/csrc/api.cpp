@@ -184,6 +184,75 @@ int attn_seq_unshard(const void* gathered, void* out, int S, int B, int H, int L
   return st;
 }
 
+int attn_query_rows_for_keys(int L, int k_first, int k_last, int mask_kind, int window,
+                             int* r_lo, int* r_hi) {
+  if (!r_lo || !r_hi || L <= 0 || k_first < 0 || k_last < k_first || k_last >= L)
+    return ATTN_ERR_INVALID;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_CAUSAL_WINDOW) return ATTN_ERR_INVALID;
+  if (has_window(mask_kind) && window < 0) return ATTN_ERR_INVALID;
+  ebh::query_rows_for_keys(L, k_first, k_last, mask_kind, window, *r_lo, *r_hi);
+  return ATTN_OK;
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int L) {
+  if (B <= 0 || H <= 0 || L <= 0) return 0;
+  return static_cast<size_t>(B) * H * L * sizeof(float);
+}
+
+int attn_bwd(const attn_params* p, const void* dout, float* dq, float* dk, float* dv,
+             void* workspace, size_t workspace_bytes, void* stream) {
+  ebh::FwdArgs a;
+  int st = validate(p, &a);
+  if (st != ATTN_OK) return st;
+  if (!p->lse || !dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID;
+  if (p->block_n != 0) return ATTN_ERR_INVALID;
+  if (p->d > 128) return ATTN_ERR_UNSUPPORTED;
+  const uint64_t rows = static_cast<uint64_t>(p->B) * p->H * p->L;
+  const uint64_t elem = p->dtype == ATTN_DTYPE_BF16 ? 2 : 4;
+  const uint64_t in_bytes = rows * p->d * elem;
+  const uint64_t g_bytes = rows * p->d * 4;
+  if (workspace_bytes < rows * 4) return ATTN_ERR_INVALID;
+  if (!aligned(dout, 16) || !aligned(dq, 4) || !aligned(dk, 4) || !aligned(dv, 4) ||
+      !aligned(workspace, 4))
+    return ATTN_ERR_MISALIGNED;
+  {  // the three gradients and the workspace must not overlap anything
+    const void* outs[4] = {dq, dk, dv, workspace};
+    const uint64_t out_sz[4] = {g_bytes, g_bytes, g_bytes, rows * 4};
+    const void* ins[6] = {p->q, p->k, p->v, p->out, dout, p->lse};
+    const uint64_t in_sz[6] = {in_bytes, in_bytes, in_bytes, in_bytes, in_bytes, rows * 4};
+    for (int x = 0; x < 4; ++x) {
+      for (int y = 0; y < 6; ++y)
+        if (overlap(outs[x], out_sz[x], ins[y], in_sz[y])) return ATTN_ERR_INVALID;
+      for (int y = x + 1; y < 4; ++y)
+        if (overlap(outs[x], out_sz[x], outs[y], out_sz[y])) return ATTN_ERR_INVALID;
+    }
+  }
+  if ((st = check_device_sm100()) != ATTN_OK) return st;
+  ebh::BwdArgs b;
+  b.q = p->q;
+  b.k = p->k;
+  b.v = p->v;
+  b.out = p->out;
+  b.dout = dout;
+  b.lse = p->lse;
+  b.D = static_cast<float*>(workspace);
+  b.dq = dq;
+  b.dk = dk;
+  b.dv = dv;
+  b.bf16 = p->dtype == ATTN_DTYPE_BF16;
+  b.B = p->B;
+  b.H = p->H;
+  b.L = p->L;
+  b.d = p->d;
+  b.scale = p->scale;
+  b.mask_kind = a.mask_kind;
+  b.window = a.window;
+  cudaError_t err = cudaSuccess;
+  st = ebh::launch_bwd(b, static_cast<cudaStream_t>(stream), &err);
+  if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
+  return st;
+}
+
 size_t attn_mha_workspace_bytes(int B, int L, int E) {
   if (B <= 0 || L <= 0 || E <= 0) return 0;
   return ebh::mha_workspace_bytes(B, L, E);

@@ -61,6 +61,25 @@ int read_device_status(int device, int reset, cudaError_t* err);
 int launch_unshard(const void* src, void* dst, int S, int BH, int Ls, int d, int elem_bytes,
                    cudaStream_t stream, cudaError_t* err);
 
+// Backward by recomputation (validated).
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* out;   // the forward's O
+  const void* dout;  // dO, same dtype as q
+  const float* lse;  // the forward's natural-log LSE
+  float* D;          // workspace: [B, H, L] row dots <dO_i, O_i>
+  float* dq;
+  float* dk;
+  float* dv;
+  bool bf16;
+  int B, H, L, d;
+  float scale;
+  int mask_kind, window;
+};
+int launch_bwd(const BwdArgs& a, cudaStream_t stream, cudaError_t* err);
+
 // The multi-head attention layer (validated).
 struct MhaArgs {
   const void* x;       // bf16 [B, L, E]

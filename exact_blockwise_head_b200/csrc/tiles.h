@@ -126,4 +126,34 @@ EBH_HD void row_allowed_cols(int L, int i, int j, int mask_kind, int window,
   c_hi = (int)hi;
 }
 
+// Query rows [r_lo, r_hi) (half-open, clipped to [0, L)) holding at least one
+// row that may attend to some key in [k_first, k_last] (inclusive, < L): the
+// rows a key block's gradients gather from.
+EBH_HD void query_rows_for_keys(int L, int k_first, int k_last, int mask_kind, int window,
+                                int& r_lo, int& r_hi) {
+  long long lo = 0, hi = L;  // half-open
+  if (mask_kind == kMaskCausal) {
+    lo = k_first;
+  } else if (mask_kind == kMaskWindow) {
+    lo = (long long)k_first - window;
+    hi = (long long)k_last + window + 1;
+  } else if (mask_kind == kMaskCausalWindow) {
+    lo = k_first;
+    hi = (long long)k_last + window + 1;
+  }
+  if (lo < 0) lo = 0;
+  if (hi > L) hi = L;
+  if (hi < lo) hi = lo;
+  r_lo = (int)lo;
+  r_hi = (int)hi;
+}
+
+// May query row i attend to key j (both < L)?
+EBH_HD bool pair_allowed(int i, int j, int mask_kind, int window) {
+  if (mask_kind == kMaskCausal) return j <= i;
+  if (mask_kind == kMaskWindow) return (long long)i - j <= window && (long long)j - i <= window;
+  if (mask_kind == kMaskCausalWindow) return j <= i && (long long)i - j <= window;
+  return true;
+}
+
 }  // namespace ebh

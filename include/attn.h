@@ -264,6 +264,31 @@ ATTN_API int attn_merge(const float* o_parts, const float* lse_parts, int num_sp
 ATTN_API int attn_fwd_splitkv_noalloc(const attn_params* p, int num_splits, void* stream);
 
 /*
+ * Backward of the forward by recomputation ("Attention optimisation
+ * strategies and practice for long-sequence inference", section 3.1;
+ * "Mosaic multi-GPU sequence-sharded attention", section 2.2): the weights
+ * P_ij = exp(scale <q_i, k_j> - lse_i) are recomputed from Q, K and the
+ * forward's LSE, never stored, and
+ *   dV_j = sum_i P_ij dO_i,  dS_ij = P_ij (<dO_i, v_j> - <dO_i, O_i>),
+ *   dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i.
+ * p describes the forward call: q, k, v and p->out (the forward's O) in
+ * p->dtype (bf16 or fp32), p->lse (the forward's LSE, required), the mask,
+ * window and scale; p->block_n must be 0.  dout: dO, [B, H, L, d] in p->dtype,
+ * 16-byte aligned.  dq, dk, dv: fp32 [B, H, L, d] outputs.  workspace:
+ * device memory of at least attn_bwd_workspace_bytes(B, H, L) bytes.  No
+ * output or the workspace may overlap any other argument.  d <= 128 (bf16:
+ * 64 or 128).  fp32 arithmetic on the CUDA cores.  Asynchronous on `stream`.
+ */
+ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int L);
+/* Host copy of the backward's rule: query rows [*r_lo, *r_hi) holding every
+ * row that may attend to some key in [k_first, k_last] (inclusive, < L).
+ * ATTN_ERR_INVALID on bad arguments. */
+ATTN_API int attn_query_rows_for_keys(int L, int k_first, int k_last, int mask_kind, int window,
+                                      int* r_lo, int* r_hi);
+ATTN_API int attn_bwd(const attn_params* p, const void* dout, float* dq, float* dk, float* dv,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * The multi-head attention layer of "Transformer multi-head attention, 8-head
  * parallel computation" (lshu.cn), sections 2.1 and 2.2:
  *   qkv = x W_qkv^T + b_qkv; q, k, v = its three E-wide thirds, each split

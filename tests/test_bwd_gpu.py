@@ -1,0 +1,89 @@
+"""Backward by recomputation on the GPU, through the C ABI, against the fp64
+oracle's gradients (which are pinned by finite differences of the forward).
+
+The GPU backward takes the forward's own O and LSE.  Bounds:
+  * fp32 inputs: normwise relative 1e-4 (the forward's fp32 bound);
+  * bf16 inputs: the backward sees the bf16 forward's rounded O (2^-9
+    relative) and its LSE (within 1e-3), which perturb D_i = <dO_i, O_i> and
+    P_ij by about 1e-3 relative; bound max|g - g*| <= 2e-2 max|g*|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import exact_blockwise_head_b200 as ebh
+from tests import gpu_helpers as G
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    G.require_gpu()
+
+
+def _run(q, k, v, g, mask, window, scale=None):
+    qd, kd, vd, gd = (t.cuda() for t in (q, k, v, g))
+    out, lse = ebh.forward(qd, kd, vd, scale=scale, mask=mask, window=window)
+    dq, dk, dv = ebh.backward(qd, kd, vd, out, lse, gd, scale=scale, mask=mask, window=window)
+    torch.cuda.synchronize()
+    assert ebh.device_status(0) == ebh.ATTN_OK
+    return [t.double().cpu().numpy() for t in (dq, dk, dv)]
+
+
+def _oracle(q, k, v, g, mask, window, scale=None):
+    import oracle
+
+    return oracle.attention_backward(G.as_f32(q), G.as_f32(k), G.as_f32(v), G.as_f32(g),
+                                     scale=scale, mask=mask, window=window)
+
+
+CASES = [
+    # (B, H, L, d, mask, window)
+    (1, 2, 300, 64, "none", 0),
+    (1, 2, 257, 128, "causal", 0),
+    (2, 1, 400, 64, "window", 37),
+    (1, 3, 333, 128, "causal_window", 50),
+    (1, 1, 1, 64, "causal", 0),
+    (1, 2, 1000, 128, "causal", 0),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: str(c).replace(" ", ""))
+def test_bf16_backward_matches_oracle(case):
+    B, H, L, d, mask, window = case
+    q, k, v = G.rand_qkv(B, H, L, d, seed=L + d + 1)
+    g = G.rand_qkv(B, H, L, d, seed=L + d + 2)[0]
+    got = _run(q, k, v, g, mask, window)
+    ref = _oracle(q, k, v, g, mask, window)
+    for name, a, b in zip(("dq", "dk", "dv"), got, ref):
+        assert np.isfinite(a).all()
+        err = np.abs(a - b).max()
+        assert err <= 2e-2 * np.abs(b).max(), f"{case} {name}: {err:.3e} vs max {np.abs(b).max():.3e}"
+
+
+@pytest.mark.parametrize("L,d,mask,window", [(200, 40, "causal", 0), (130, 17, "window", 9),
+                                             (256, 128, "none", 0), (99, 64, "causal_window", 20)])
+def test_f32_backward_matches_oracle(L, d, mask, window):
+    q, k, v = G.rand_qkv(1, 2, L, d, seed=L * 3 + d, dtype="f32")
+    g = G.rand_qkv(1, 2, L, d, seed=L * 3 + d + 1, dtype="f32")[0]
+    got = _run(q, k, v, g, mask, window, scale=0.2)
+    ref = _oracle(q, k, v, g, mask, window, scale=0.2)
+    for name, a, b in zip(("dq", "dk", "dv"), got, ref):
+        norm = np.abs(a - b).max() / np.abs(b).max()
+        assert norm <= 1e-4, f"f32 {L} {d} {mask} {name}: normwise {norm:.3e}"
+
+
+def test_backward_invariants_on_gpu():
+    """Constant V -> dQ = dK = 0; a common key shift -> sum_j dK_j = 0;
+    sum_j dV_j = sum_i dO_i (rows of P sum to one)."""
+    B, H, L, d = 1, 2, 500, 64
+    q, k, _ = G.rand_qkv(B, H, L, d, seed=3, dtype="f32")
+    g = G.rand_qkv(B, H, L, d, seed=4, dtype="f32")[0]
+    c = torch.randn(B, H, 1, d).expand(B, H, L, d).contiguous()
+    dq, dk, _ = _run(q, k, c, g, "causal", 0)
+    assert np.abs(dq).max() <= 1e-4 and np.abs(dk).max() <= 1e-4
+    v = G.rand_qkv(B, H, L, d, seed=5, dtype="f32")[2]
+    dq, dk, dv = _run(q, k, v, g, "causal", 0)
+    assert np.abs(dk.sum(axis=2)).max() <= 1e-3
+    assert np.abs(dv.sum(axis=2) - g.double().numpy().sum(axis=2)).max() <= 1e-3

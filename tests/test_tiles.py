@@ -61,3 +61,19 @@ def test_bad_tile_arguments():
         ebh.kv_tile_range(10, 0, 10)
     with pytest.raises(ebh.AttnError):
         ebh.kv_tile_class(10, 0, 3, 0, "window", -1)
+
+
+@pytest.mark.parametrize("L,mask,window", [c for c in CASES if c[0] <= 300])
+def test_query_rows_for_keys_match_dense_mask(L, mask, window):
+    """The rows a key block's gradients gather from (backward)."""
+    M = _dense(L, mask, window)
+    for kt in (1, 32, 128):
+        for k_first in range(0, L, kt):
+            k_last = min(k_first + kt - 1, L - 1)
+            lo, hi = ebh.query_rows_for_keys(L, k_first, k_last, mask, window)
+            rows = np.nonzero(M[:, k_first:k_last + 1].any(axis=1))[0]
+            if len(rows):
+                assert lo <= rows.min() and rows.max() < hi, (L, mask, window, k_first)
+                assert lo == rows.min() and hi == rows.max() + 1, (L, mask, window, k_first)
+            else:
+                assert lo == hi
