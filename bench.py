@@ -308,6 +308,33 @@ def sweep_layer(ebh, torch, B=4, L=2048, E=512, H=8, steps=10):
             "flops": "8 B L E^2 (projections) + 4 B H L^2 d (attention)"}
 
 
+def sweep_backward(ebh, torch, name="causal_bf16_L8192_d128", steps=3):
+    """The backward (dQ, dK, dV by recomputation) on one workload.
+    Algorithmic FLOPs: 10 d per allowed pair (the recomputed S, dP, and the
+    three gradient products, 2 d each)."""
+    w = ebh.WORKLOADS[name]
+    g = torch.Generator(device="cuda").manual_seed(w.seed)
+    shape = (w.B, w.H, w.L, w.d)
+    q, k, v, do = ((torch.randn(shape, device="cuda", generator=g) * w.std).to(torch.bfloat16)
+                   for _ in range(4))
+    out, lse = ebh.forward(q, k, v, mask=w.mask, window=w.window)
+    dq, dk, dv = (torch.empty(shape, device="cuda", dtype=torch.float32) for _ in range(3))
+    ws = torch.empty(w.B * w.H * w.L * 4, dtype=torch.uint8, device="cuda")
+
+    def fn():
+        ebh.backward(q, k, v, out, lse, do, mask=w.mask, window=w.window, dq=dq, dk=dk, dv=dv,
+                     workspace=ws)
+
+    fn()
+    torch.cuda.synchronize()
+    ms = time_gpu(fn, steps, torch.cuda.current_stream())
+    avg = sum(ms) / len(ms)
+    flops = 10.0 * w.d * w.B * w.H * allowed_pairs(w.L, w.mask, w.window)
+    return {"workload": name, "ms": round(avg, 3), "tflops": round(flops / avg / 1e9, 2),
+            "kernels": "row dots, dK/dV per key tile, dQ per query tile (CUDA cores, fp32)",
+            "l2": "inputs larger than L2"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -466,6 +493,7 @@ def main():
         del qe, ke, ve
         line["other_workloads_kernel_only"] = sweep_other(ebh, torch, others)
         line["mha_layer"] = sweep_layer(ebh, torch)
+        line["backward"] = sweep_backward(ebh, torch)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, q, k, v, args.cpu_seconds)
     if world > 1:
