@@ -91,3 +91,45 @@ def test_gloo_ranks_return_their_rows_of_the_definition(world, mask, window):
     l = np.concatenate([x[2] for x in got], axis=2)
     assert np.abs(o - full_o).max() <= 1e-12
     assert np.abs(l - full_l).max() <= 1e-12
+
+
+def _failing_rank_main(rank, world, port, result):
+    """Rank 1 fails before the gather; rank 0 must get an error from its
+    collective (the peer left, or the short process-group timeout ran out)
+    instead of waiting for good."""
+    import datetime
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=10))
+    B, H, Ls, d = 1, 1, 8, 4
+    x = torch.zeros(B, H, Ls, d)
+    if rank == 1:
+        result.put((rank, "left"))
+        result.close()
+        result.join_thread()  # the message is out before the process ends
+        os._exit(0)  # leaves between steps, with no collective in flight
+    try:
+        seqpar.forward(x, x, x, mask="causal", ops=_CpuOps())
+        result.put((rank, "no error"))
+    except Exception as e:  # noqa: BLE001 - any backend error is the detection
+        result.put((rank, type(e).__name__))
+    result.close()
+    result.join_thread()
+    os._exit(0)
+
+
+def test_a_rank_that_leaves_is_detected_by_the_others():
+    ctx = mp.get_context("spawn")
+    result = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_rank_main, args=(r, 2, port, result)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict(result.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert got[1] == "left"
+    assert got[0] != "no error", got
