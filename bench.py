@@ -682,10 +682,7 @@ def reference_arm(args, w, world, rank):
         rows = step()
         for i in rows:
             i = int(i)
-            n = w.L if w.mask == "none" else (i + 1 if w.mask == "causal" else
-                                              min(w.L - 1, i + w.window) - max(0, i - w.window)
-                                              + 1)
-            flops += 4 * w.d * n
+            flops += 4 * w.d * allowed_pairs_rows(w.L, i, i + 1, w.mask, w.window)
     dt = time.perf_counter() - t0
     value = flops / dt / 1e12
     line = {
