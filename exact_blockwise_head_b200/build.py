@@ -1,11 +1,13 @@
 """Build libebh_attn.so in-tree with nvcc for sm_100a.
 
-    python -m exact_blockwise_head_b200.build [--force] [--verbose]
+    python -m exact_blockwise_head_b200.build [--force] [--verbose] [--trace|--debug]
 
 The library is the C ABI of include/attn.h: api.cpp (validation, dispatch),
-attn_sm100.cu (tcgen05 bf16 kernel), attn_f32.cu (fp32 CUDA-core kernel).
-The CUDA runtime is linked statically, so the .so needs only libcuda at run
-time.
+attn_sm100.cu (tcgen05 bf16 kernel), attn_f32.cu (fp32 CUDA-core kernel), the
+split-KV merge, sequence-shard layout, multi-head layer and backward kernels.
+The CUDA runtime is linked statically; cuBLASLt (the layer's projections) is
+linked dynamically.  Two variants build beside it: libebh_attn_trace.so
+(pipeline timestamps) and libebh_attn_debug.so (bounds-checked stores).
 """
 from __future__ import annotations
 
@@ -19,6 +21,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libebh_attn.so")
 TRACE_LIB = os.path.join(PKG, "libebh_attn_trace.so")
+DEBUG_LIB = os.path.join(PKG, "libebh_attn_debug.so")
 SOURCES = ["api.cpp", "attn_sm100.cu", "attn_f32.cu", "attn_merge.cu", "noalloc.cu",
            "seqpar.cu", "mha.cu", "attn_bwd.cu"]
 HEADERS = ["kernels.h", "sm100_ptx.cuh", "tiles.h"]
@@ -39,31 +42,36 @@ def _inputs():
     return files
 
 
-def is_stale() -> bool:
-    if not os.path.exists(LIB):
+def is_stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(f) > t for f in _inputs())
 
 
 def build(force: bool = False, verbose: bool = False, trace: bool = False,
-          defines=(), out: str | None = None) -> str:
+          defines=(), out: str | None = None, debug: bool = False) -> str:
     """Compile every source into libebh_attn.so (skipped when up to date).
 
     trace=True builds the profiling variant libebh_attn_trace.so, whose
     tensor-core kernel records pipeline timestamps for CTA 0 (read back with
-    attn_pipeline_trace_read).  `defines` are extra -D flags; `out` overrides
-    the output path.
+    attn_pipeline_trace_read).  debug=True builds libebh_attn_debug.so, whose
+    tensor-core kernel checks every global store against the array's extent
+    and counts refusals (attn_debug_bounds_violations).  `defines` are extra
+    -D flags; `out` overrides the output path.
     """
-    target = out or (TRACE_LIB if trace else LIB)
-    if not force and not defines and out is None and target == LIB and not is_stale():
-        return LIB
+    target = out or (TRACE_LIB if trace else (DEBUG_LIB if debug else LIB))
+    if not force and not defines and out is None and target in (LIB, DEBUG_LIB) and \
+            not is_stale(target):
+        return target
     tmp = target + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC,-O3,-fvisibility=hidden", "-cudart", "static",
            "-I", INCLUDE, "-I", CSRC, "-o", tmp]
     if trace:
         cmd.append("-DEBH_PIPELINE_TRACE")
+    if debug:
+        cmd.append("-DEBH_BOUNDS_CHECK")
     cmd += [f"-D{d}" for d in defines]
     if verbose:
         cmd += ["-Xptxas", "-v"]
@@ -76,4 +84,4 @@ def build(force: bool = False, verbose: bool = False, trace: bool = False,
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
-                trace="--trace" in sys.argv))
+                trace="--trace" in sys.argv, debug="--debug" in sys.argv))

@@ -109,6 +109,21 @@ __device__ unsigned long long g_pipeline_trace[20][kTraceLen];
   } while (0)
 #endif
 
+// Bounds-checking builds (-DEBH_BOUNDS_CHECK, the debug library): every
+// global store of the kernel checks its element index against the array's
+// extent; an index outside is counted in g_bounds_violations and the store is
+// skipped (no trap).  Release builds compile the check away.
+#ifdef EBH_BOUNDS_CHECK
+__device__ unsigned long long g_bounds_violations;
+__device__ __forceinline__ bool in_bounds(size_t idx, size_t n) {
+  if (idx < n) return true;
+  atomicAdd(&g_bounds_violations, 1ull);
+  return false;
+}
+#else
+__device__ __forceinline__ bool in_bounds(size_t, size_t) { return true; }
+#endif
+
 template <int D, int BN>
 struct Cfg {
   static_assert(D == 64 || D == 128, "head dim");
@@ -184,7 +199,7 @@ __device__ __forceinline__ TileWork decode_tile(int u, int t, const Params& p) {
     qp = u % p.nqp;
   }
   w.q_first = qp * kUnitRows + t * kBM;
-  w.valid = w.q_first < p.L;
+  w.valid = w.q_first < p.L && in_bounds(static_cast<size_t>(w.bh), static_cast<size_t>(p.BH));
   w.q_last = min(w.q_first + kBM - 1, p.L - 1);
   w.lo = w.hi = 0;
   if (w.valid) {
@@ -937,12 +952,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                                           __uint_as_float(o[4 * m + 1]) * inv_a);
           const uint32_t vb = pack_bf16x2(__uint_as_float(o[4 * m + 2]) * inv_b,
                                           __uint_as_float(o[4 * m + 3]) * inv_b);
-          if (ok_a) dst_a[col2] = va;
-          if (ok_b) dst_b[col2] = vb;
+          if (ok_a && in_bounds((static_cast<size_t>(w.bh) * p.L + row_a) * (D / 2) + col2,
+                                static_cast<size_t>(p.BH) * p.L * (D / 2)))
+            dst_a[col2] = va;
+          if (ok_b && in_bounds((static_cast<size_t>(w.bh) * p.L + row_b) * (D / 2) + col2,
+                                static_cast<size_t>(p.BH) * p.L * (D / 2)))
+            dst_b[col2] = vb;
         }
         if (t0 == 0 && p.lse != nullptr) {
-          if (ok_a) p.lse[static_cast<size_t>(w.bh) * p.L + row_a] = lse_a;
-          if (ok_b) p.lse[static_cast<size_t>(w.bh) * p.L + row_b] = lse_b;
+          const size_t n_lse = static_cast<size_t>(p.BH) * p.L;
+          if (ok_a && in_bounds(static_cast<size_t>(w.bh) * p.L + row_a, n_lse))
+            p.lse[static_cast<size_t>(w.bh) * p.L + row_a] = lse_a;
+          if (ok_b && in_bounds(static_cast<size_t>(w.bh) * p.L + row_b, n_lse))
+            p.lse[static_cast<size_t>(w.bh) * p.L + row_b] = lse_b;
         }
       } else {
         // split-KV partial: fp32 O normalised within the split, and its LSE
@@ -954,16 +976,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int m = 0; m < D / 8; ++m) {
           const int col2 = 4 * m + t0;
-          if (ok_a)
+          const size_t n_part = static_cast<size_t>(p.num_splits) * p.BH * p.L * (D / 2);
+          if (ok_a && in_bounds((head * p.L + row_a) * (D / 2) + col2, n_part))
             dst_a[col2] = make_float2(__uint_as_float(o[4 * m]) * inv_a,
                                       __uint_as_float(o[4 * m + 1]) * inv_a);
-          if (ok_b)
+          if (ok_b && in_bounds((head * p.L + row_b) * (D / 2) + col2, n_part))
             dst_b[col2] = make_float2(__uint_as_float(o[4 * m + 2]) * inv_b,
                                       __uint_as_float(o[4 * m + 3]) * inv_b);
         }
         if (t0 == 0) {
-          if (ok_a) p.lse_part[head * p.L + row_a] = lse_a;
-          if (ok_b) p.lse_part[head * p.L + row_b] = lse_b;
+          const size_t n_lpart = static_cast<size_t>(p.num_splits) * p.BH * p.L;
+          if (ok_a && in_bounds(head * p.L + row_a, n_lpart)) p.lse_part[head * p.L + row_a] = lse_a;
+          if (ok_b && in_bounds(head * p.L + row_b, n_lpart)) p.lse_part[head * p.L + row_b] = lse_b;
         }
       }
       EBH_TRACE(kEvEpilogueDone, 0);
@@ -1157,6 +1181,22 @@ int read_device_status(int device, int reset, cudaError_t* err) {
 }
 
 }  // namespace ebh
+
+#ifdef EBH_BOUNDS_CHECK
+// Bounds-checking builds only: the number of refused out-of-range stores
+// since the last reset.
+extern "C" __attribute__((visibility("default"))) long long attn_debug_bounds_violations(
+    int reset) {
+  unsigned long long n = 0;
+  if (cudaMemcpyFromSymbol(&n, ebh::g_bounds_violations, sizeof(n)) != cudaSuccess) return -1;
+  if (reset) {
+    const unsigned long long zero = 0;
+    if (cudaMemcpyToSymbol(ebh::g_bounds_violations, &zero, sizeof(zero)) != cudaSuccess)
+      return -1;
+  }
+  return static_cast<long long>(n);
+}
+#endif
 
 #ifdef EBH_PIPELINE_TRACE
 // Profiling builds only: copy out / clear the pipeline trace of CTA 0.
