@@ -39,7 +39,8 @@ EXPORTED = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ex", "attn_strerror", "attn_la
             "attn_kv_tile_class", "attn_kv_full_range", "attn_splitkv_workspace_bytes",
             "attn_fwd_splitkv", "attn_merge", "attn_abi_version", "attn_fwd_splitkv_noalloc",
             "attn_fwd_rows", "attn_seq_unshard", "attn_mha_workspace_bytes", "attn_mha_fwd",
-            "attn_bwd_workspace_bytes", "attn_bwd", "attn_query_rows_for_keys")
+            "attn_bwd_workspace_bytes", "attn_bwd", "attn_query_rows_for_keys",
+            "attn_fwd_strided")
 
 
 class AttnParams(ctypes.Structure):
@@ -123,6 +124,8 @@ def _load():
             lib.attn_fwd_splitkv.argtypes = [ctypes.POINTER(AttnParams), i, vp, ctypes.c_size_t, vp]
             lib.attn_fwd_splitkv_noalloc.argtypes = [ctypes.POINTER(AttnParams), i, vp]
             lib.attn_fwd_rows.argtypes = [ctypes.POINTER(AttnParams), i, i, vp]
+            lib.attn_fwd_strided.argtypes = [ctypes.POINTER(AttnParams),
+                                             ctypes.POINTER(ctypes.c_int64), vp]
             lib.attn_seq_unshard.argtypes = [vp, vp, i, i, i, i, i, i, vp]
             lib.attn_mha_workspace_bytes.argtypes = [i, i, i]
             lib.attn_bwd_workspace_bytes.argtypes = [i, i, i]
@@ -203,6 +206,62 @@ def forward(q, k, v, scale=None, mask="none", window=0, block_n=0, out=None, lse
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_ex")
     return out, (lse if want_lse else None)
+
+
+def forward_strided(q, k, v, B, H, L, d, strides, scale=None, mask="none", window=0,
+                    block_n=0, out=None, lse=None, want_lse=True, stream=None):
+    """bf16 forward on tensors in any (row, head, batch) layout: element
+    (b, h, i, c) of q is at q.data_ptr() + 2 (b s[2] + h s[1] + i s[0] + c) with
+    s = strides[0] (and strides[1..3] for k, v, out; element units).  q, k, v
+    and out are CUDA bf16 tensors (views are fine); out is required.  lse, when
+    wanted, is dense [B, H, L].  Returns (out, lse)."""
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        if t is None or not t.is_cuda or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be a bf16 CUDA tensor")
+    if mask not in MASK_KINDS:
+        raise ValueError(f"mask must be one of {sorted(MASK_KINDS)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if want_lse and lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    p = AttnParams()
+    p.dtype = ATTN_DTYPE_BF16
+    p.q, p.k, p.v, p.out = q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr()
+    p.lse = lse.data_ptr() if (want_lse and lse is not None) else None
+    p.B, p.H, p.L, p.d = B, H, L, d
+    p.scale = float(scale)
+    p.mask_kind = MASK_KINDS[mask]
+    p.window = int(window)
+    p.block_n = int(block_n)
+    p.wait_timeout_ns = 0
+    flat = (ctypes.c_int64 * 12)(*[int(x) for s3 in strides for x in s3])
+    with torch.cuda.device(q.device):
+        st = _load().attn_fwd_strided(ctypes.byref(p), flat, _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_strided")
+    return out, (lse if want_lse else None)
+
+
+def forward_bshd(q, k, v, scale=None, mask="none", window=0, block_n=0, out=None, lse=None,
+                 want_lse=True, stream=None):
+    """forward() for the [B, L, H, d] layout (sequence before heads): q, k, v
+    and the returned out are [B, L, H, d] bf16; lse is [B, H, L]."""
+    import torch
+
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share one [B, L, H, d] shape")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    B, L, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    s = (H * d, d, L * H * d)
+    return forward_strided(q, k, v, B, H, L, d, (s, s, s, s), scale=scale, mask=mask,
+                           window=window, block_n=block_n, out=out, lse=lse, want_lse=want_lse,
+                           stream=stream)
 
 
 def forward_rows(q, k, v, q_offset, scale=None, mask="none", window=0, block_n=0, out=None,

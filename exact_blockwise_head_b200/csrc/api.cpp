@@ -38,7 +38,9 @@ bool overlap(const void* a, uint64_t na, const void* b, uint64_t nb) {
 }
 
 // Validation common to both paths; fills `out` with the normalised problem.
-int validate(const attn_params* p, ebh::FwdArgs* out) {
+// check_overlap = false leaves the aliasing checks to a caller that knows the
+// tensors' real extents (strided layouts).
+int validate(const attn_params* p, ebh::FwdArgs* out, bool check_overlap = true) {
   if (p == nullptr) return ATTN_ERR_INVALID;
   if (p->dtype != ATTN_DTYPE_BF16 && p->dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID;
   if (!p->q || !p->k || !p->v || !p->out) return ATTN_ERR_INVALID;
@@ -58,11 +60,11 @@ int validate(const attn_params* p, ebh::FwdArgs* out) {
   const uint64_t rows = static_cast<uint64_t>(p->B) * p->H * p->L;
   const uint64_t tensor_bytes = rows * p->d * elem;
   const uint64_t lse_bytes = rows * 4;
-  if (overlap(p->out, tensor_bytes, p->q, tensor_bytes) ||
-      overlap(p->out, tensor_bytes, p->k, tensor_bytes) ||
-      overlap(p->out, tensor_bytes, p->v, tensor_bytes))
+  if (check_overlap && (overlap(p->out, tensor_bytes, p->q, tensor_bytes) ||
+                        overlap(p->out, tensor_bytes, p->k, tensor_bytes) ||
+                        overlap(p->out, tensor_bytes, p->v, tensor_bytes)))
     return ATTN_ERR_INVALID;
-  if (p->lse && (overlap(p->lse, lse_bytes, p->q, tensor_bytes) ||
+  if (check_overlap && p->lse && (overlap(p->lse, lse_bytes, p->q, tensor_bytes) ||
                  overlap(p->lse, lse_bytes, p->k, tensor_bytes) ||
                  overlap(p->lse, lse_bytes, p->v, tensor_bytes) ||
                  overlap(p->lse, lse_bytes, p->out, tensor_bytes)))
@@ -133,6 +135,37 @@ int attn_fwd_ex(const attn_params* p, void* stream) {
   st = p->dtype == ATTN_DTYPE_BF16
            ? ebh::launch_fwd_bf16_sm100(a, static_cast<cudaStream_t>(stream), &err)
            : ebh::launch_fwd_f32(a, static_cast<cudaStream_t>(stream), &err);
+  if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
+  return st;
+}
+
+int attn_fwd_strided(const attn_params* p, const int64_t* strides, void* stream) {
+  if (p == nullptr || strides == nullptr) return ATTN_ERR_INVALID;
+  if (p->dtype != ATTN_DTYPE_BF16) return ATTN_ERR_UNSUPPORTED;
+  ebh::FwdArgs a;
+  int st = validate(p, &a, false);
+  if (st != ATTN_OK) return st;
+  // extent in bytes of each tensor: one past its last element
+  uint64_t ext[4];
+  for (int x = 0; x < 4; ++x) {
+    const int64_t* s3 = strides + 3 * x;
+    for (int y = 0; y < 3; ++y)
+      if (s3[y] <= 0 || s3[y] % 8 != 0 || s3[y] > (int64_t(1) << 38)) return ATTN_ERR_INVALID;
+    if (s3[0] < p->d) return ATTN_ERR_INVALID;
+    ext[x] = (static_cast<uint64_t>(p->B - 1) * s3[2] + static_cast<uint64_t>(p->H - 1) * s3[1] +
+              static_cast<uint64_t>(p->L - 1) * s3[0] + p->d) * 2;
+    for (int y = 0; y < 3; ++y) a.stride[x][y] = s3[y];
+  }
+  const void* in[3] = {p->q, p->k, p->v};
+  const uint64_t lse_bytes = static_cast<uint64_t>(p->B) * p->H * p->L * 4;
+  for (int x = 0; x < 3; ++x) {
+    if (overlap(p->out, ext[3], in[x], ext[x])) return ATTN_ERR_INVALID;
+    if (p->lse && overlap(p->lse, lse_bytes, in[x], ext[x])) return ATTN_ERR_INVALID;
+  }
+  if (p->lse && overlap(p->lse, lse_bytes, p->out, ext[3])) return ATTN_ERR_INVALID;
+  if ((st = check_device_sm100()) != ATTN_OK) return st;
+  cudaError_t err = cudaSuccess;
+  st = ebh::launch_fwd_bf16_sm100(a, static_cast<cudaStream_t>(stream), &err);
   if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
   return st;
 }

@@ -24,6 +24,9 @@ struct FwdArgs {
   // rows (0: Lk = L), and query row i sits at key position q_shift + i.
   int Lk = 0;
   int q_shift = 0;
+  // Element strides (row, head, batch) of q, k, v and out on the bf16 path;
+  // all zero: dense [B, H, rows, d].
+  long long stride[4][3] = {};
   // split-KV partial mode (bf16 path): when o_part is set, the keys are cut
   // into num_splits runs of split_keys (a multiple of block_n) and the kernel
   // writes fp32 partial O [S,B,H,L,d] and partial LSE [S,B,H,L] instead of

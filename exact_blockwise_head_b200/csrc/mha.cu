@@ -8,8 +8,10 @@
 //   context = softmax(q k^T / sqrt(d) + mask) v, transposed back to [B, L, E]
 //   y = context W_out^T + b_out        (one Linear(E, E))
 // The two projections are plain GEMMs and run in cuBLASLt (bf16 operands,
-// fp32 accumulation, the bias added in its epilogue); the head split and
-// merge are this file's kernels; the attention is attn_fwd_ex's kernel.
+// fp32 accumulation, the bias added in its epilogue).  The attention kernel
+// reads q, k and v straight out of the projection's [B, L, 3, H, d] output
+// through strided tensor maps and writes the context in [B, L, H, d], so the
+// head split and merge cost no pass of their own.
 #include <cublasLt.h>
 #include <cuda_runtime.h>
 
@@ -22,55 +24,7 @@
 namespace ebh {
 namespace {
 
-constexpr int kLayoutThreads = 256;
 constexpr size_t kLtWorkspace = size_t(32) << 20;
-
-// qkv [B, L, 3, H, d] (rows of the Linear output) -> q, k, v [B, H, L, d],
-// moved in 16-byte chunks (d * 2 bytes is a multiple of 16 for d in {64, 128}).
-__global__ void __launch_bounds__(kLayoutThreads)
-    split_heads_kernel(const uint4* __restrict__ qkv, uint4* __restrict__ q, uint4* __restrict__ k,
-                       uint4* __restrict__ v, int B, int L, int H, int d_chunks) {
-  const long long per_tensor = static_cast<long long>(B) * H * L * d_chunks;
-  const long long total = 3 * per_tensor;
-  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-       e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    // source index: ((b L + l) 3 + which) H d_chunks + h d_chunks + c
-    const int c = static_cast<int>(e % d_chunks);
-    long long r = e / d_chunks;
-    const int h = static_cast<int>(r % H);
-    r /= H;
-    const int which = static_cast<int>(r % 3);
-    const long long bl = r / 3;
-    const int l = static_cast<int>(bl % L);
-    const int b = static_cast<int>(bl / L);
-    uint4* dst = which == 0 ? q : (which == 1 ? k : v);
-    dst[((static_cast<long long>(b) * H + h) * L + l) * d_chunks + c] = qkv[e];
-  }
-}
-
-// o [B, H, L, d] -> context [B, L, H, d] (= [B, L, E]).
-__global__ void __launch_bounds__(kLayoutThreads)
-    merge_heads_kernel(const uint4* __restrict__ o, uint4* __restrict__ ctx, int B, int L, int H,
-                       int d_chunks) {
-  const long long total = static_cast<long long>(B) * L * H * d_chunks;
-  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-       e += static_cast<long long>(gridDim.x) * blockDim.x) {
-    // destination index: ((b L + l) H + h) d_chunks + c
-    const int c = static_cast<int>(e % d_chunks);
-    long long r = e / d_chunks;
-    const int h = static_cast<int>(r % H);
-    const long long bl = r / H;
-    const int l = static_cast<int>(bl % L);
-    const int b = static_cast<int>(bl / L);
-    ctx[e] = o[((static_cast<long long>(b) * H + h) * L + l) * d_chunks + c];
-  }
-}
-
-unsigned grid_for(long long units) {
-  long long blocks = (units + kLayoutThreads - 1) / kLayoutThreads;
-  if (blocks > 148LL * 64) blocks = 148LL * 64;
-  return static_cast<unsigned>(blocks < 1 ? 1 : blocks);
-}
 
 cublasLtHandle_t lt_handle(int device, cublasStatus_t* st) {
   static std::mutex mu;
@@ -140,8 +94,8 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 size_t mha_workspace_bytes(int B, int L, int E) {
   const size_t act = static_cast<size_t>(B) * L * E * 2;  // one [B, L, E] bf16 tensor
-  // qkv (3) + q, k, v (3) + o (1) + context (1), then the cuBLASLt workspace
-  return align256(3 * act) + 3 * align256(act) + 2 * align256(act) + kLtWorkspace;
+  // qkv (3) + context (1), then the cuBLASLt workspace
+  return align256(3 * act) + align256(act) + kLtWorkspace;
 }
 
 int launch_mha(const MhaArgs& a, void* workspace, cudaStream_t stream, cudaError_t* err,
@@ -151,16 +105,8 @@ int launch_mha(const MhaArgs& a, void* workspace, cudaStream_t stream, cudaError
   const int d = a.E / a.H;
   const size_t act = static_cast<size_t>(a.B) * a.L * a.E * 2;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  void* qkv = ws;
+  uint16_t* qkv = reinterpret_cast<uint16_t*>(ws);
   ws += align256(3 * act);
-  void* q = ws;
-  ws += align256(act);
-  void* k = ws;
-  ws += align256(act);
-  void* v = ws;
-  ws += align256(act);
-  void* o = ws;
-  ws += align256(act);
   void* ctx = ws;
   ws += align256(act);
   void* lt_ws = ws;
@@ -178,17 +124,12 @@ int launch_mha(const MhaArgs& a, void* workspace, cudaStream_t stream, cudaError
     *lt_status = 1;
     return ATTN_ERR_CUDA;
   }
-  const int d_chunks = d * 2 / 16;
-  split_heads_kernel<<<grid_for(3LL * M * a.E / 8), kLayoutThreads, 0, stream>>>(
-      static_cast<const uint4*>(qkv), static_cast<uint4*>(q), static_cast<uint4*>(k),
-      static_cast<uint4*>(v), a.B, a.L, a.H, d_chunks);
-  if ((*err = cudaGetLastError()) != cudaSuccess) return ATTN_ERR_CUDA;
-
+  // q, k, v: the three E-wide thirds of each qkv row, head h at columns h d
   FwdArgs f;
-  f.q = q;
-  f.k = k;
-  f.v = v;
-  f.out = o;
+  f.q = qkv;
+  f.k = qkv + a.E;
+  f.v = qkv + 2 * a.E;
+  f.out = ctx;
   f.lse = nullptr;
   f.B = a.B;
   f.H = a.H;
@@ -199,13 +140,17 @@ int launch_mha(const MhaArgs& a, void* workspace, cudaStream_t stream, cudaError
   f.window = a.window;
   f.block_n = 128;
   f.timeout_ns = a.timeout_ns;
+  const long long E3 = 3LL * a.E;
+  for (int x = 0; x < 3; ++x) {
+    f.stride[x][0] = E3;
+    f.stride[x][1] = d;
+    f.stride[x][2] = E3 * a.L;
+  }
+  f.stride[3][0] = a.E;  // context [B, L, H, d]
+  f.stride[3][1] = d;
+  f.stride[3][2] = static_cast<long long>(a.E) * a.L;
   const int st = launch_fwd_bf16_sm100(f, stream, err);
   if (st != ATTN_OK) return st;
-
-  merge_heads_kernel<<<grid_for(static_cast<long long>(M) * a.E / 8), kLayoutThreads, 0,
-                       stream>>>(static_cast<const uint4*>(o), static_cast<uint4*>(ctx), a.B,
-                                 a.L, a.H, d_chunks);
-  if ((*err = cudaGetLastError()) != cudaSuccess) return ATTN_ERR_CUDA;
   if (!linear_bf16(h, ctx, a.w_out, a.b_out, a.y, M, a.E, a.E, lt_ws, stream)) {
     *lt_status = 2;
     return ATTN_ERR_CUDA;

@@ -131,6 +131,21 @@ typedef struct attn_params {
 ATTN_API int attn_fwd_ex(const attn_params* p, void* stream);
 
 /*
+ * bf16 forward on tensors in any (row, head, batch) layout with contiguous
+ * head dim: element (b, h, i, c) of q sits at
+ *   q + b strides[2] + h strides[1] + i strides[0] + c
+ * and likewise k (strides[3..5]), v (strides[6..8]) and out (strides[9..11]),
+ * all in elements.  For example [B, L, H, d] tensors have strides (H d, d,
+ * L H d), and the thirds of a fused [B, L, 3, H, d] projection have (3 H d,
+ * d, 3 L H d) from bases 0, H d and 2 H d.  Every stride is positive, a
+ * multiple of 8 (16 bytes; the tensor-memory-access copy rule) and, for rows,
+ * at least d.  lse stays dense [B, H, L] fp32 or NULL.  out may not overlap q,
+ * k, v or lse; q, k, v may overlap each other.  Other arguments and errors as
+ * attn_fwd_ex (bf16 only).
+ */
+ATTN_API int attn_fwd_strided(const attn_params* p, const int64_t* strides, void* stream);
+
+/*
  * Forward for a block of query rows placed inside a longer key sequence:
  * q, out are [B, H, L, d] with L = p->L query rows, k, v are [B, H, kv_len, d],
  * lse is [B, H, L]; query row i sits at key position q_offset + i, and the
@@ -298,11 +313,13 @@ ATTN_API int attn_bwd(const attn_params* p, const void* dout, float* dq, float* 
  * output feature j; rows [0, E) make q, [E, 2E) k, [2E, 3E) v); w_out: bf16
  * [E, E]; b_qkv [3E] and b_out [E]: bf16 or NULL.  d in {64, 128}; every
  * pointer 16-byte aligned.  The projections run in cuBLASLt (fp32
- * accumulation, bias in its epilogue, bf16 results); the head split and merge
- * and the attention run in this library's kernels.  q, k, v, the attention
- * output and the context are bf16 in `workspace`: device memory, 256-byte
- * aligned, at least attn_mha_workspace_bytes(B, L, E) bytes, disjoint from
- * the other arguments.  On a cuBLASLt failure the call returns ATTN_ERR_CUDA
+ * accumulation, bias in its epilogue, bf16 results); the attention runs in
+ * this library's kernel, reading each head's q, k, v straight from the
+ * projection output and writing the context in [B, L, H, d] (the head split
+ * and merge are its strides).  The projection output and the context are
+ * bf16 in `workspace`: device memory, 256-byte aligned, at least
+ * attn_mha_workspace_bytes(B, L, E) bytes, disjoint from the other
+ * arguments.  On a cuBLASLt failure the call returns ATTN_ERR_CUDA
  * and attn_last_cuda_error() returns -(1 for the first projection, 2 for the
  * second).  Asynchronous on `stream`.
  */
