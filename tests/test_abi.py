@@ -134,3 +134,52 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(ebh, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(ImportError):
         ebh.library()
+
+
+def test_newer_entry_points_validate_before_any_device_work(lib):
+    """Argument errors of the split-KV, offset-rows, strided, backward,
+    unshard and no-allocation calls come back as status codes on a machine
+    without a GPU (validation runs before anything touches a device)."""
+    p = _params(L=256, d=64)
+    # offset rows: rows must fit inside the keys
+    assert lib.attn_fwd_rows(ctypes.byref(p), 100, 0, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_fwd_rows(ctypes.byref(p), 300, -1, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_fwd_rows(ctypes.byref(p), 300, 45, None) == ebh.ATTN_ERR_INVALID
+    # strided: strides positive, multiples of 8 elements, rows at least d
+    good = [128, 64, 256 * 128]
+    for bad in ([132, 64, 256 * 128], [32, 64, 256 * 128], [128, 0, 256 * 128],
+                [128, 64, -8]):
+        flat = (ctypes.c_int64 * 12)(*(bad + good * 3))
+        assert lib.attn_fwd_strided(ctypes.byref(p), flat, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_fwd_strided(ctypes.byref(p), None, None) == ebh.ATTN_ERR_INVALID
+    pf = _params(dtype=ebh.ATTN_DTYPE_F32, block_n=0)
+    flat = (ctypes.c_int64 * 12)(*(good * 4))
+    assert lib.attn_fwd_strided(ctypes.byref(pf), flat, None) == ebh.ATTN_ERR_UNSUPPORTED
+    # split-KV: split count and workspace
+    assert lib.attn_fwd_splitkv(ctypes.byref(p), 0, None, 0, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_fwd_splitkv(ctypes.byref(p), 65, None, 0, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_fwd_splitkv(ctypes.byref(p), 2, None, 0, None) == ebh.ATTN_ERR_INVALID
+    # no-allocation split-KV: a problem whose partials exceed the scratch
+    big = _params(B=1, H=32, L=8192, d=128)
+    assert lib.attn_fwd_splitkv_noalloc(ctypes.byref(big), 2, None) == ebh.ATTN_ERR_SCRATCH_LIMIT
+    # backward: lse, gradients and workspace are required; block_n must be 0
+    ws, g = 1 << 30, 1 << 31
+    assert lib.attn_bwd(ctypes.byref(_params(lse=0)), g, g, g + (1 << 26), g + (2 << 26), ws,
+                        1 << 20, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_bwd(ctypes.byref(_params(block_n=64)), g, g + (1 << 26), g + (2 << 26),
+                        g + (3 << 26), ws, 1 << 20, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_bwd(ctypes.byref(p), g, g + (1 << 26), g + (2 << 26), g + (3 << 26), ws, 4,
+                        None) == ebh.ATTN_ERR_INVALID
+    # the gradients may not overlap one another
+    assert lib.attn_bwd(ctypes.byref(p), g, g + (1 << 26), g + (1 << 26), g + (3 << 26), ws,
+                        1 << 20, None) == ebh.ATTN_ERR_INVALID
+    # unshard: element size and overlap
+    assert lib.attn_seq_unshard(1 << 20, 1 << 28, 2, 1, 1, 8, 64, 3, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_seq_unshard(1 << 20, 1 << 20, 2, 1, 1, 8, 64, 2, None) == ebh.ATTN_ERR_INVALID
+    # the host copy of the backward's tile rule
+    lo, hi = ctypes.c_int(), ctypes.c_int()
+    assert lib.attn_query_rows_for_keys(10, 3, 2, 1, 0, ctypes.byref(lo), ctypes.byref(hi)) == \
+        ebh.ATTN_ERR_INVALID
+    assert lib.attn_query_rows_for_keys(10, 2, 3, 1, 0, ctypes.byref(lo), ctypes.byref(hi)) == \
+        ebh.ATTN_OK
+    assert (lo.value, hi.value) == (2, 10)
