@@ -68,3 +68,22 @@ def test_splitkv_and_rows_stores_stay_in_bounds(debug_library):
     _no_violations(debug_library)
     G.check_bf16(o2.double().cpu().numpy(), l2.double().cpu().numpy(),
                  ref_o[:, :, off:off + 500], ref_l[:, :, off:off + 500], "debug rows")
+
+
+def test_strided_stores_stay_in_bounds(debug_library):
+    """[B, L, H, d] tensors with padded rows: the strided epilogue's stores."""
+    B, H, L, d = 2, 3, 333, 64
+    row = H * d + 64  # each sequence position padded by 64 elements
+    g = torch.Generator().manual_seed(11)
+    bufs = [torch.randn(B, L, row, generator=g).to(torch.bfloat16).cuda() for _ in range(3)]
+    out = torch.zeros(B, L, row, dtype=torch.bfloat16, device="cuda")
+    s = (row, d, L * row)
+    for mask, window in (("causal", 0), ("window", 50)):
+        ebh.forward_strided(bufs[0], bufs[1], bufs[2], B, H, L, d, (s, s, s, s), mask=mask,
+                            window=window, out=out)
+        _no_violations(debug_library)
+        heads = [t[..., :H * d].reshape(B, L, H, d).transpose(1, 2).cpu() for t in bufs]
+        ref_o, _ = G.oracle_full(*heads, mask=mask, window=window)
+        got = out[..., :H * d].reshape(B, L, H, d).transpose(1, 2).double().cpu().numpy()
+        assert np.abs(got - ref_o).max() <= G.BF16_OUT_ATOL
+        assert (out[..., H * d:] == 0).all()
