@@ -185,8 +185,10 @@ class ClockSampler:
                 "samples": len(s)}
 
 
-def cpu_baseline(w, q, k, v, budget_s: float):
-    """Time the fp64 oracle, as it stands, on a bounded sample of query rows."""
+def cpu_baseline(w, q, k, v, budget_s: float, gpu_out=None, gpu_lse=None):
+    """Time the fp64 oracle, as it stands, on a bounded sample of query rows.
+    When the GPU's O and LSE for the same inputs are given, the sampled rows
+    are also compared with them (the parity of the timed run)."""
     import numpy as np
 
     import oracle
@@ -197,25 +199,20 @@ def cpu_baseline(w, q, k, v, budget_s: float):
     rng = np.random.default_rng(1234)
 
     def rows_flops(row_idx):
-        total = 0
-        for i in row_idx:
-            i = int(i)
-            if w.mask == "none":
-                n = w.L
-            elif w.mask == "causal":
-                n = i + 1
-            else:
-                n = min(w.L - 1, i + w.window) - max(0, i - w.window) + 1
-            total += 4 * w.d * n
-        return total
+        return sum(4 * w.d * allowed_pairs_rows(w.L, int(i), int(i) + 1, w.mask, w.window)
+                   for i in row_idx)
+
+    last = {}
 
     def run(n):
         bh = rng.integers(0, BH, size=n)
         rows = rng.integers(0, w.L, size=n)
         t0 = time.perf_counter()
-        oracle.attention_rows(qf, kf, vf, bh, rows, mask=w.mask, window=w.window,
-                              nthreads=threads)
-        return time.perf_counter() - t0, rows_flops(rows)
+        o, l = oracle.attention_rows(qf, kf, vf, bh, rows, mask=w.mask, window=w.window,
+                                     nthreads=threads)
+        dt = time.perf_counter() - t0
+        last.update(bh=bh, rows=rows, o=o, l=l)
+        return dt, rows_flops(rows)
 
     n = max(threads, 8)
     dt, fl = run(n)
@@ -224,10 +221,19 @@ def cpu_baseline(w, q, k, v, budget_s: float):
         dt, fl = run(n)
     n_final = max(1, int(n * budget_s / max(dt, 1e-6)))
     dt, fl = run(n_final)
-    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n_final} random query rows of {w.name} (fp64 C oracle, "
-                      f"{threads} threads, {dt:.1f} s)",
-            "rows_per_s": n_final / dt, "tokens_per_s_extrapolated": n_final / dt}
+    res = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+           "sample": f"{n_final} random query rows of {w.name} (fp64 C oracle, "
+                     f"{threads} threads, {dt:.1f} s)",
+           "rows_per_s": n_final / dt, "tokens_per_s_extrapolated": n_final / dt}
+    if gpu_out is not None:
+        o = gpu_out.reshape(BH, w.L, w.d)[last["bh"], last["rows"]].astype(np.float64)
+        l = gpu_lse.reshape(BH, w.L)[last["bh"], last["rows"]].astype(np.float64)
+        res["parity_on_sample"] = {
+            "rows": int(n_final),
+            "max_abs_err_out": float(np.abs(o - last["o"]).max()),
+            "max_abs_err_lse": float(np.abs(l - last["l"]).max()),
+            "bounds": "2e-2 (out), 1e-3 (lse)"}
+    return res
 
 
 def time_gpu(fn, steps, stream, flush=None):
@@ -480,6 +486,10 @@ def main():
     peaks, peak_kind = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     per_launch_ms = sum(ms) / len(ms)
+    ms_sorted = sorted(ms)
+    pct = lambda f: ms_sorted[min(len(ms_sorted) - 1, int(f * len(ms_sorted)))]  # noqa: E731
+    # algorithmic bytes: Q, K, V read once, O and LSE written once
+    alg_bytes = 4 * qd.numel() * 2 + lse.numel() * 4
     achieved = algorithmic_flops(w) / (per_launch_ms * 1e-3) / 1e12
     line = {
         "metric": METRIC,
@@ -515,6 +525,9 @@ def main():
                 "pipelined": "copy-in, forward and copy-out on three streams; step i+1's "
                              "copies overlap step i"},
         "gpu_launches": args.steps,
+        "step_ms": {"median": round(pct(0.5), 5), "p10": round(pct(0.1), 5),
+                    "p90": round(pct(0.9), 5)},
+        "hbm_gbs_algorithmic": round(alg_bytes / (pct(0.5) * 1e-3) / 1e9, 1),
         "clocks": clk.summary(),
         "context_only": CONTEXT,
     }
@@ -528,7 +541,9 @@ def main():
         line["mha_layer"] = sweep_layer(ebh, torch)
         line["backward"] = sweep_backward(ebh, torch)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, q, k, v, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(w, q, k, v, args.cpu_seconds,
+                                            gpu_out=out.float().cpu().numpy(),
+                                            gpu_lse=lse.float().cpu().numpy())
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
