@@ -185,6 +185,18 @@ class ClockSampler:
                 "samples": len(s)}
 
 
+def executed_tile_flops(ebh, w, block_n: int, rows: int = 128) -> int:
+    """FLOPs of the tiles the forward runs: every key tile of every query
+    tile's range at full size, masked lanes and ragged tails included.  Set
+    beside the algorithmic FLOPs it shows how much of the tensor work the
+    masks throw away."""
+    tiles = 0
+    for q0 in range(0, w.L, rows):
+        lo, hi = ebh.kv_tile_range(w.L, q0, min(w.L, q0 + rows) - 1, w.mask, w.window, block_n)
+        tiles += hi - lo
+    return 4 * rows * block_n * w.d * tiles * w.B * w.H
+
+
 def cpu_baseline(w, q, k, v, budget_s: float, gpu_out=None, gpu_lse=None):
     """Time the fp64 oracle, as it stands, on a bounded sample of query rows.
     When the GPU's O and LSE for the same inputs are given, the sampled rows
@@ -491,6 +503,9 @@ def main():
     # algorithmic bytes: Q, K, V read once, O and LSE written once
     alg_bytes = 4 * qd.numel() * 2 + lse.numel() * 4
     achieved = algorithmic_flops(w) / (per_launch_ms * 1e-3) / 1e12
+    executed = executed_tile_flops(ebh, w, args.block_n or 128)
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS.get("hbm_gbs", 6650.0)))
+    hbm_gbs = alg_bytes / (pct(0.5) * 1e-3) / 1e9
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -518,7 +533,9 @@ def main():
                      "frac_of_sustained": round(
                          achieved / float(peaks.get("bf16_tflops_sustained", 1400.0)), 4),
                      "traffic": traffic_for(w.name),
-                     "flops_per_launch": algorithmic_flops(w)},
+                     "flops_per_launch": algorithmic_flops(w),
+                     "executed_tile_flops_per_launch": executed,
+                     "executed_tflops": round(executed / (per_launch_ms * 1e-3) / 1e12, 1)},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "ms_per_step": round(float(e2e_t.item()), 4),
@@ -527,7 +544,9 @@ def main():
         "gpu_launches": args.steps,
         "step_ms": {"median": round(pct(0.5), 5), "p10": round(pct(0.1), 5),
                     "p90": round(pct(0.9), 5)},
-        "hbm_gbs_algorithmic": round(alg_bytes / (pct(0.5) * 1e-3) / 1e9, 1),
+        "hbm": {"gbs_algorithmic": round(hbm_gbs, 1), "frac_of_measured": round(hbm_gbs / hbm_peak, 4),
+                "frac_of_spec_8000": round(hbm_gbs / 8000.0, 4),
+                "bytes_per_launch": alg_bytes},
         "clocks": clk.summary(),
         "context_only": CONTEXT,
     }
