@@ -292,6 +292,18 @@ def sweep_other(ebh, torch, names, steps=5, warmup=3):
         res[name] = {"ms": round(avg, 4), "tflops": round(fl / avg / 1e9, 1),
                      "tokens_per_s": round(w.B * w.L / avg * 1e3, 1),
                      "l2": "flushed between steps" if small else "inputs larger than L2"}
+        if small:
+            # also 100 launches back to back, inputs left in L2 (one event pair)
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(100):
+                fn()
+            t1.record(stream)
+            t1.synchronize()
+            b2b = t0.elapsed_time(t1) / 100
+            res[name]["back_to_back_100"] = {"ms": round(b2b, 4),
+                                             "tflops": round(fl / b2b / 1e9, 1)}
         del q, k, v, out, lse, flush_buf
     return res
 
