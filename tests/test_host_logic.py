@@ -39,6 +39,24 @@ def test_row_range_pairs_add_up(mask, window):
         assert bench.allowed_pairs_rows(L, a, b, mask, window) == int(M[a:b].sum())
 
 
+@pytest.mark.parametrize("L", [1, 100, 128, 300, 1000])
+@pytest.mark.parametrize("mask,window", [("none", 0), ("causal", 0), ("window", 40),
+                                         ("window", 300), ("causal_window", 129)])
+@pytest.mark.parametrize("block_n", [64, 128])
+def test_executed_tile_flops_counts_tiles_with_an_allowed_pair(L, mask, window, block_n):
+    """The bench's executed-tile count: every (128-row query tile, key block)
+    pair holding at least one allowed (i, j), at full tile size."""
+    M = np.array(dense_mask(L, mask, window))
+    tiles = 0
+    for q0 in range(0, L, 128):
+        for k0 in range(0, L, block_n):
+            tiles += bool(M[q0:q0 + 128, k0:k0 + block_n].any())
+    w = ebh.WORKLOADS["causal_bf16_L8192_d128"].with_(B=2, H=3, L=L, d=64, mask=mask,
+                                                       window=window)
+    assert bench.executed_tile_flops(ebh, w, block_n) == 4 * 128 * block_n * 64 * tiles * 6
+    assert bench.executed_tile_flops(ebh, w, block_n) >= bench.algorithmic_flops(w)
+
+
 @pytest.mark.parametrize("total,world", [(0, 1), (1, 1), (7, 2), (32, 8), (5, 8), (100, 3)])
 def test_shard_range_partitions(total, world):
     seen = []
