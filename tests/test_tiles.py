@@ -31,7 +31,7 @@ for L in (1, 2, 63, 64, 65, 127, 128, 129, 200, 256, 300):
 @pytest.mark.parametrize("L,mask,window", CASES)
 def test_range_and_class_match_dense_mask(L, mask, window):
     M = _dense(L, mask, window)
-    for bn, rows in ((64, 128), (128, 128), (32, 64)):
+    for bn, rows in ((64, 128), (128, 128), (256, 128), (32, 64)):
         for q_first in range(0, L, rows):
             q_last = min(q_first + rows - 1, L - 1)
             lo, hi = ebh.kv_tile_range(L, q_first, q_last, mask, window, bn)
