@@ -93,6 +93,21 @@ def allowed_pairs_rows(L: int, a: int, b: int, mask: str, window: int) -> int:
     return total
 
 
+def bench_config(w, block_n: int, world: int, l2_note: str) -> dict:
+    """The `config` of the bench line; both arms print the same keys."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
+            "mask": w.mask, "window": w.window,
+            "block_n": block_n or 128, "heads_per_gpu": w.B * w.H,
+            "global_heads": w.B * w.H * world, "parallelism": f"heads sharded x{world}",
+            "l2": l2_note}
+
+
+def l2_note_for(w) -> str:
+    if 3 * w.B * w.H * w.L * w.d * 2 < 126e6:
+        return "L2 flushed between steps (256 MB write, outside the events)"
+    return "inputs larger than L2 (126 MB)"
+
+
 def algorithmic_flops(w) -> float:
     return 4.0 * w.d * w.B * w.H * allowed_pairs(w.L, w.mask, w.window)
 
@@ -137,7 +152,7 @@ class ClockSampler:
         0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.0005):
         self.samples = []
         self.reasons = 0
         self.period = period_s
@@ -236,7 +251,9 @@ def cpu_baseline(w, q, k, v, budget_s: float, gpu_out=None, gpu_lse=None):
     res = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
            "sample": f"{n_final} random query rows of {w.name} (fp64 C oracle, "
                      f"{threads} threads, {dt:.1f} s)",
-           "rows_per_s": n_final / dt, "tokens_per_s_extrapolated": n_final / dt}
+           "rows_per_s": n_final / dt,
+           # a token is one query position through every head: H rows
+           "tokens_per_s_extrapolated": n_final / dt / w.H}
     if gpu_out is not None:
         o = gpu_out.reshape(BH, w.L, w.d)[last["bh"], last["rows"]].astype(np.float64)
         l = gpu_lse.reshape(BH, w.L)[last["bh"], last["rows"]].astype(np.float64)
@@ -416,12 +433,11 @@ def main():
     lse = torch.empty((w.B, w.H, w.L), device="cuda", dtype=torch.float32)
     stream = torch.cuda.current_stream()
     inputs_bytes = 3 * qd.numel() * 2
-    l2_note = "inputs larger than L2 (126 MB)"
+    l2_note = l2_note_for(w)
     flush = None
     if inputs_bytes < 126e6:
         flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
         flush = lambda: flush_buf.zero_()  # noqa: E731
-        l2_note = "L2 flushed between steps (256 MB write, outside the events)"
 
     def step():
         ebh.forward(qd, kd, vd, mask=w.mask, window=w.window, block_n=args.block_n, out=out,
@@ -532,11 +548,7 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) inputs of the workload's shape)",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d,
-                   "mask": w.mask, "window": w.window,
-                   "block_n": args.block_n or 128, "heads_per_gpu": w.B * w.H,
-                   "global_heads": w.B * w.H * world, "parallelism": f"heads sharded x{world}",
-                   "l2": l2_note},
+        "config": bench_config(w, args.block_n, world, l2_note),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)"
@@ -548,6 +560,11 @@ def main():
                      "flops_per_launch": algorithmic_flops(w),
                      "executed_tile_flops_per_launch": executed,
                      "executed_tflops": round(executed / (per_launch_ms * 1e-3) / 1e12, 1)},
+        "target": {"what": "causal bf16 L=8192 d=128 forward at >= 60% of the 2.25 PFLOP/s "
+                           "dense bf16 spec", "tflops": 0.6 * SPEC_BF16_TFLOPS,
+                   "frac_of_spec_2250": round(achieved / SPEC_BF16_TFLOPS, 4),
+                   "met": bool(w.name == DEFAULT_WORKLOAD
+                               and achieved >= 0.6 * SPEC_BF16_TFLOPS)},
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "ms_per_step": round(float(e2e_t.item()), 4),
@@ -713,22 +730,25 @@ def reference_arm(args, w, world, rank):
     rng = np.random.default_rng(99)
     rows_per_step = 32 * max(threads, 1)
 
-    def step():
+    def draw():
         bh = rng.integers(0, w.B * w.H, size=rows_per_step)
         rows = rng.integers(0, w.L, size=rows_per_step)
+        return bh, rows
+
+    def step(sample):
+        bh, rows = sample
         oracle.attention_rows(qf, kf, vf, bh, rows, mask=w.mask, window=w.window,
                               nthreads=threads)
-        return rows
 
     for _ in range(args.warmup):
-        step()
-    flops = 0
+        step(draw())
+    # every step's rows and their FLOPs are fixed before the clock starts
+    samples = [draw() for _ in range(args.steps)]
+    flops = sum(4 * w.d * allowed_pairs_rows(w.L, int(i), int(i) + 1, w.mask, w.window)
+                for _, rows in samples for i in rows)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        rows = step()
-        for i in rows:
-            i = int(i)
-            flops += 4 * w.d * allowed_pairs_rows(w.L, i, i + 1, w.mask, w.window)
+    for sample in samples:
+        step(sample)
     dt = time.perf_counter() - t0
     value = flops / dt / 1e12
     line = {
@@ -736,8 +756,7 @@ def reference_arm(args, w, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "mask": w.mask,
-                   "window": w.window},
+        "config": bench_config(w, args.block_n, world, l2_note_for(w)),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"{rows_per_step} random query rows per step of {w.name}"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,

@@ -122,6 +122,19 @@ int check_device_sm100() {
 
 namespace ebh {
 void set_last_cuda_error(cudaError_t e) { g_last_cuda_error = static_cast<int>(e); }
+
+int splitkv_check(const attn_params* p, int num_splits, int* runs, int* run_blocks) {
+  FwdArgs a;
+  int st = validate(p, &a);
+  if (st != ATTN_OK) return st;
+  if (p->dtype != ATTN_DTYPE_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (num_splits < 1 || num_splits > kMaxSplits) return ATTN_ERR_INVALID;
+  // whole key blocks per run; the last run may be shorter
+  const int nkv = (a.L + a.block_n - 1) / a.block_n;
+  *run_blocks = (nkv + num_splits - 1) / num_splits;
+  *runs = (nkv + *run_blocks - 1) / *run_blocks;
+  return ATTN_OK;
+}
 }  // namespace ebh
 
 extern "C" {
@@ -445,16 +458,12 @@ size_t attn_splitkv_workspace_bytes(int B, int H, int L, int d, int num_splits) 
 
 int attn_fwd_splitkv(const attn_params* p, int num_splits, void* workspace,
                      size_t workspace_bytes, void* stream) {
-  ebh::FwdArgs a;
-  int st = validate(p, &a);
+  int splits = 0, split_blocks = 0;
+  int st = ebh::splitkv_check(p, num_splits, &splits, &split_blocks);
   if (st != ATTN_OK) return st;
-  if (p->dtype != ATTN_DTYPE_BF16) return ATTN_ERR_UNSUPPORTED;
-  if (num_splits < 1 || num_splits > ebh::kMaxSplits) return ATTN_ERR_INVALID;
-  // whole key blocks per split; the last split may be shorter
-  const int nkv = (a.L + a.block_n - 1) / a.block_n;
-  const int split_blocks = (nkv + num_splits - 1) / num_splits;
-  const int splits = (nkv + split_blocks - 1) / split_blocks;
   if (splits == 1) return attn_fwd_ex(p, stream);
+  ebh::FwdArgs a;
+  if ((st = validate(p, &a)) != ATTN_OK) return st;
   const size_t need = attn_splitkv_workspace_bytes(a.B, a.H, a.L, a.d, splits);
   if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_INVALID;
   if (!aligned(workspace, 256)) return ATTN_ERR_MISALIGNED;

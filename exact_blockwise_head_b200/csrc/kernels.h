@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "attn.h"
+
 namespace ebh {
 
 // One validated forward problem (see include/attn.h for the meaning).
@@ -100,6 +102,12 @@ size_t mha_workspace_bytes(int B, int L, int E);
 // On ATTN_ERR_CUDA, *err holds a CUDA error or *lt_status a cuBLASLt failure.
 int launch_mha(const MhaArgs& a, void* workspace, cudaStream_t stream, cudaError_t* err,
                int* lt_status);
+
+// Every argument check of attn_fwd_splitkv except those on the workspace
+// (defined in api.cpp).  On ATTN_OK, *runs is the number of key runs the call
+// will use and *run_blocks the key blocks per run (the last run may be
+// shorter); one run means the call is a plain forward and needs no workspace.
+int splitkv_check(const attn_params* p, int num_splits, int* runs, int* run_blocks);
 
 // Records e as this thread's attn_last_cuda_error() (defined in api.cpp).
 void set_last_cuda_error(cudaError_t e);

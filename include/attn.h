@@ -262,12 +262,18 @@ ATTN_API int attn_merge(const float* o_parts, const float* lse_parts, int num_sp
  *   - Limit: the partials of the runs actually used must fit, i.e.
  *     attn_splitkv_workspace_bytes(B, H, L, d, runs) <= ATTN_NOALLOC_SCRATCH_BYTES
  *     (at d=128 about 64K rows of B*H*L*runs); otherwise it returns
- *     ATTN_ERR_SCRATCH_LIMIT and enqueues nothing.  With one run it is
- *     attn_fwd_ex and the scratch is not touched.
+ *     ATTN_ERR_SCRATCH_LIMIT and enqueues nothing.  Every other argument is
+ *     checked first, exactly as attn_fwd_splitkv checks it, so an invalid
+ *     call gets ATTN_ERR_INVALID / UNSUPPORTED / MISALIGNED whatever its
+ *     size.  With one run it is attn_fwd_ex and the scratch is not touched.
  *   - Set-up: the first call on a device (the current device) looks up the
- *     scratch's device address with cudaGetSymbolAddress and keeps it; make
- *     that first call before any stream capture on that device.  A failed
- *     look-up returns ATTN_ERR_CUDA.
+ *     scratch's device address with cudaGetSymbolAddress, in the CUDA
+ *     context current on the calling thread, and keeps it with that
+ *     context's unique ID.  A later call reuses the address only while the
+ *     same context is current; after cudaDeviceReset, or with another
+ *     context made current on the device, the next call looks it up again
+ *     (that call is again a set-up call).  Make every set-up call before any
+ *     stream capture on that device.  A failed look-up returns ATTN_ERR_CUDA.
  *   - Concurrency: every call on a device uses the same scratch, so calls
  *     whose work may overlap on the GPU (unordered streams, several host
  *     threads) race and corrupt each other's results; order them, e.g. on

@@ -160,8 +160,26 @@ def test_newer_entry_points_validate_before_any_device_work(lib):
     assert lib.attn_fwd_splitkv(ctypes.byref(p), 65, None, 0, None) == ebh.ATTN_ERR_INVALID
     assert lib.attn_fwd_splitkv(ctypes.byref(p), 2, None, 0, None) == ebh.ATTN_ERR_INVALID
     # no-allocation split-KV: a problem whose partials exceed the scratch
-    big = _params(B=1, H=32, L=8192, d=128)
+    gb = 1 << 30  # tensors 1 GiB apart: the 64 MiB ones below do not overlap
+    far = dict(q=gb, k=2 * gb, v=3 * gb, out=4 * gb, lse=5 * gb)
+    big = _params(B=1, H=32, L=8192, d=128, **far)
     assert lib.attn_fwd_splitkv_noalloc(ctypes.byref(big), 2, None) == ebh.ATTN_ERR_SCRATCH_LIMIT
+    # ... but every other argument is checked before the scratch limit: a call
+    # too big for the scratch that is also invalid reports what is invalid
+    assert lib.attn_fwd_splitkv_noalloc(ctypes.byref(_params(B=1, H=32, L=8192, d=128, **{**far, "q": 0})), 2,
+                                        None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_fwd_splitkv_noalloc(ctypes.byref(_params(B=1, H=32, L=8192, d=96, **far)), 2,
+                                        None) == ebh.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_fwd_splitkv_noalloc(
+        ctypes.byref(_params(B=1, H=32, L=8192, d=128, dtype=ebh.ATTN_DTYPE_F32, block_n=0, **far)),
+        2,
+        None) == ebh.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_fwd_splitkv_noalloc(ctypes.byref(_params(B=1, H=32, L=8192, d=128,
+                                                             block_n=96, **far)), 2,
+                                        None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_fwd_splitkv_noalloc(ctypes.byref(big), 0, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_fwd_splitkv_noalloc(ctypes.byref(big), 65, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_fwd_splitkv_noalloc(None, 2, None) == ebh.ATTN_ERR_INVALID
     # backward: lse, gradients and workspace are required; block_n must be 0
     ws, g = 1 << 30, 1 << 31
     assert lib.attn_bwd(ctypes.byref(_params(lse=0)), g, g, g + (1 << 26), g + (2 << 26), ws,
