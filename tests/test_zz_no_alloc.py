@@ -124,8 +124,9 @@ def test_no_alloc_matches_workspace_call_and_oracle_twice(shape, mask, window, s
 def test_no_alloc_allocates_nothing():
     """After its first (set-up) call, the entry point changes neither torch's
     allocator peak nor the device's free memory."""
-    B, H, L, d, splits, block_n = 1, 4, 2048, 128, 8, 0
+    B, H, L, d, splits, block_n = 1, 2, 2048, 128, 8, 0
     assert _runs(L, splits, block_n) == 8
+    assert ebh.splitkv_workspace_bytes(B, H, L, d, 8) <= ebh.NOALLOC_SCRATCH_BYTES
     q, k, v = (t.cuda() for t in G.rand_qkv(B, H, L, d, seed=5))
     out = torch.empty_like(q)
     lse = torch.empty(B, H, L, dtype=torch.float32, device="cuda")
