@@ -377,8 +377,15 @@ def sweep_backward(ebh, torch, name="causal_bf16_L8192_d128", steps=3):
     ms = time_gpu(fn, steps, torch.cuda.current_stream())
     avg = sum(ms) / len(ms)
     flops = 10.0 * w.d * w.B * w.H * allowed_pairs(w.L, w.mask, w.window)
+    peaks, _ = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     return {"workload": name, "ms": round(avg, 3), "tflops": round(flops / avg / 1e9, 2),
-            "kernels": "row dots, dK/dV per key tile, dQ per query tile (CUDA cores, fp32)",
+            "frac_of_measured_bf16": round(flops / avg / 1e9 / peak, 4),
+            "flops": "10 d per allowed pair (S, dP, dV, dK, dQ); the dQ kernel recomputes S "
+                     "and dP, so the tensor cores execute 14 d per pair",
+            "kernels": "row dots (CUDA cores); dK/dV per 128-key tile and dQ per 128-query "
+                       "tile on the tensor cores (tcgen05 MMAs, fp32 accumulators in tensor "
+                       "memory)",
             "l2": "inputs larger than L2"}
 
 

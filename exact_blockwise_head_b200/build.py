@@ -24,7 +24,7 @@ TRACE_LIB = os.path.join(PKG, "libebh_attn_trace.so")
 DEBUG_LIB = os.path.join(PKG, "libebh_attn_debug.so")
 SOURCES = ["api.cpp", "attn_sm100.cu", "attn_f32.cu", "attn_merge.cu", "noalloc.cu",
            "seqpar.cu", "mha.cu", "attn_bwd.cu"]
-HEADERS = ["kernels.h", "sm100_ptx.cuh", "tiles.h"]
+HEADERS = ["kernels.h", "sm100_ptx.cuh", "tiles.h", "attn_bwd_sm100.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

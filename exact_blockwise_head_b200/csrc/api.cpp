@@ -52,7 +52,8 @@ int validate(const attn_params* p, ebh::FwdArgs* out, bool check_overlap = true)
     return ATTN_ERR_INVALID;
   if (has_window(p->mask_kind) && p->window < 0) return ATTN_ERR_INVALID;
   if (p->dtype == ATTN_DTYPE_BF16) {
-    if (p->block_n != 0 && p->block_n != 64 && p->block_n != 128) return ATTN_ERR_INVALID;
+    if (p->block_n != 0 && p->block_n != 64 && p->block_n != 128 && p->block_n != 256)
+      return ATTN_ERR_INVALID;
   } else if (p->block_n != 0) {
     return ATTN_ERR_INVALID;
   }

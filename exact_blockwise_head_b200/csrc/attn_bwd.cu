@@ -246,6 +246,17 @@ int launch_bwd_dtype(const BwdArgs& a, cudaStream_t stream, cudaError_t* err) {
 
 int launch_bwd(const BwdArgs& a, cudaStream_t stream, cudaError_t* err) {
   *err = cudaSuccess;
+  if (a.bf16 && (a.d == 64 || a.d == 128)) {
+    // D on the CUDA cores (one warp per row), the five products on the
+    // tensor cores
+    const long long rows = static_cast<long long>(a.B) * a.H * a.L;
+    if ((rows + 7) / 8 > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+    bwd_rowdot_kernel<__nv_bfloat16><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(a.out), static_cast<const __nv_bfloat16*>(a.dout), a.D,
+        rows, a.d);
+    if ((*err = cudaGetLastError()) != cudaSuccess) return ATTN_ERR_CUDA;
+    return launch_bwd_sm100(a, stream, err);
+  }
   return a.bf16 ? launch_bwd_dtype<__nv_bfloat16>(a, stream, err)
                 : launch_bwd_dtype<float>(a, stream, err);
 }

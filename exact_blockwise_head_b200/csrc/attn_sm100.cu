@@ -47,18 +47,29 @@ namespace ebh {
 namespace {
 
 constexpr int kBM = 128;          // query rows per Q tile (= tensor-memory lanes)
-constexpr int kNQ = 2;            // Q tiles per work unit
-constexpr int kUnitRows = kBM * kNQ;
 constexpr int kSoftmaxWarps = 8;   // per Q tile: two per tensor-memory sub-partition
 constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
-constexpr int kThreads = (kNQ * kSoftmaxWarps + 4) * 32;  // + producer, MMA, 2 idle
-constexpr int kProducerWarp = kNQ * kSoftmaxWarps;
-constexpr int kMmaWarp = kProducerWarp + 1;
-constexpr int kLaunchRegs = 96;    // 65536 / 640 rounded down to a multiple of 8
-constexpr int kSoftmaxRegs = 104;
-constexpr int kOtherRegs = 64;
-static_assert(kSoftmaxRegs * kNQ * kSoftmaxThreads + kOtherRegs * 128 <= kLaunchRegs * kThreads,
-              "register split exceeds the launch allocation");
+
+// Work-unit shape per key-block size.  With 64- and 128-key blocks a unit is
+// two 128-row Q tiles that share the K/V stream (S_0 | S_1 | O_0 | O_1 fill
+// the 512 tensor-memory columns at d = 128); with 256-key blocks one Q tile's
+// S (256 columns) and O (d columns) already take 384, so a unit is one Q tile.
+template <int BN>
+struct Layout {
+  static constexpr int kNQ = BN == 256 ? 1 : 2;  // Q tiles per work unit
+  static constexpr int kUnitRows = kBM * kNQ;
+  static constexpr int kThreads = (kNQ * kSoftmaxWarps + 4) * 32;  // + producer, MMA, 2 idle
+  static constexpr int kProducerWarp = kNQ * kSoftmaxWarps;
+  static constexpr int kMmaWarp = kProducerWarp + 1;
+  // 65536 / kThreads rounded down to a multiple of 8
+  static constexpr int kLaunchRegs = (65536 / kThreads) / 8 * 8;
+  // softmax: a BN/2-wide half row block per thread plus its packed bf16 copy
+  static constexpr int kSoftmaxRegs = kNQ == 2 ? 104 : 208;
+  static constexpr int kOtherRegs = 64;
+  static_assert(kSoftmaxRegs * kNQ * kSoftmaxThreads + kOtherRegs * 128 <=
+                    kLaunchRegs * kThreads,
+                "register split exceeds the launch allocation");
+};
 // Tuning knobs of the softmax arithmetic.  kPolyEvery: one column group of
 // eight in kPolyEvery takes its exponentials from a polynomial on the FMA pipe
 // instead of the MUFU pipe (tiles without masked elements only; 0 = none).
@@ -127,13 +138,18 @@ __device__ __forceinline__ bool in_bounds(size_t, size_t) { return true; }
 template <int D, int BN>
 struct Cfg {
   static_assert(D == 64 || D == 128, "head dim");
-  static_assert(BN == 64 || BN == 128, "key block");
+  static_assert(BN == 64 || BN == 128 || BN == 256, "key block");
+  static constexpr int kNQ = Layout<BN>::kNQ;
   static constexpr int kDChunks = D / 64;            // 128-byte (64 x bf16) column chunks
   static constexpr int kQTileBytes = kBM * D * 2;
   static constexpr int kKVTileBytes = BN * D * 2;
-  static constexpr int kStages = kKVTileBytes >= 32768 ? 4 : 8;
+  static constexpr int kStages = kKVTileBytes >= 65536 ? 2 : (kKVTileBytes >= 32768 ? 4 : 8);
   static constexpr int kSmemQ = kNQ * kQTileBytes;
   static constexpr int kSmemKV = kStages * kKVTileBytes;
+  // epilogue staging: one 16-row x 64-column bf16 box (128-byte swizzle) per
+  // softmax warp, written by the warp and stored by TMA
+  static constexpr int kOBoxBytes = 16 * 128;
+  static constexpr int kSmemO = kNQ * kSoftmaxWarps * kOBoxBytes;
   // barrier indices
   static constexpr int kBarQFull = 0;                  // [kNQ]
   static constexpr int kBarQEmpty = kBarQFull + kNQ;   // [kNQ]
@@ -146,11 +162,12 @@ struct Cfg {
   static constexpr int kBarTok = kBarOEmpty + kNQ;        // [kNQ]
   static constexpr int kBarDrain = kBarTok + kNQ;
   static constexpr int kNumBars = kBarDrain + 1;
-  static constexpr int kSmemBytes = 1024 + kSmemQ + kSmemKV + 8 * kNumBars + 16;
-  static constexpr int kTmemNeed = 2 * BN + 2 * D;
+  static constexpr int kSmemBytes = 1024 + kSmemQ + kSmemKV + kSmemO + 8 * kNumBars + 16;
+  static constexpr int kTmemNeed = kNQ * BN + kNQ * D;
   static constexpr int kTmemCols = kTmemNeed <= 256 ? 256 : 512;
   static constexpr int kColS = 0;            // + t * BN
-  static constexpr int kColO = 2 * BN;       // + t * D
+  static constexpr int kColO = kNQ * BN;     // + t * D
+  static_assert(kTmemNeed <= 512, "tensor memory budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -201,8 +218,9 @@ __device__ __forceinline__ TileWork decode_tile(int u, int t, const Params& p) {
     w.bh = u / p.nqp;
     qp = u % p.nqp;
   }
-  w.q_first = qp * kUnitRows + t * kBM;
-  w.valid = w.q_first < p.L && in_bounds(static_cast<size_t>(w.bh), static_cast<size_t>(p.BH));
+  w.q_first = qp * Layout<BN>::kUnitRows + t * kBM;
+  w.valid = t < Layout<BN>::kNQ && w.q_first < p.L &&
+            in_bounds(static_cast<size_t>(w.bh), static_cast<size_t>(p.BH));
   w.q_last = min(w.q_first + kBM - 1, p.L - 1);
   w.lo = w.hi = 0;
   if (w.valid) {
@@ -222,8 +240,8 @@ __device__ __forceinline__ TileWork decode_tile(int u, int t, const Params& p) {
 
 struct Unit {
   int bh;
-  bool valid[kNQ];
-  int q_first[kNQ], lo[kNQ], hi[kNQ];
+  bool valid[2];  // per Q tile of the unit (a one-tile unit leaves [1] invalid)
+  int q_first[2], lo[2], hi[2];
   int ulo, uhi;  // union of the two key-block ranges
 };
 
@@ -233,7 +251,7 @@ __device__ __forceinline__ Unit decode_unit(int u, const Params& p) {
   w.ulo = 0x7fffffff;
   w.uhi = 0;
 #pragma unroll
-  for (int t = 0; t < kNQ; ++t) {
+  for (int t = 0; t < 2; ++t) {
     const TileWork tw = decode_tile<BN>(u, t, p);
     w.bh = tw.bh;
     w.valid[t] = tw.valid;
@@ -286,7 +304,9 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 // Load / fence half a score row block: BN/2 keys = BN/16 column groups.
 template <int BN>
 __device__ __forceinline__ void tmem_ld_half(uint32_t taddr, uint32_t* r) {
-  if constexpr (BN == 128) {
+  if constexpr (BN == 256) {
+    tmem_ld_16x256b_x16(taddr, r);
+  } else if constexpr (BN == 128) {
     tmem_ld_16x256b_x8(taddr, r);
   } else {
     tmem_ld_16x256b_x4(taddr, r);
@@ -294,7 +314,9 @@ __device__ __forceinline__ void tmem_ld_half(uint32_t taddr, uint32_t* r) {
 }
 template <int BN>
 __device__ __forceinline__ void reg_fence_half(uint32_t* r) {
-  if constexpr (BN == 128) {
+  if constexpr (BN == 256) {
+    reg_fence64(r);
+  } else if constexpr (BN == 128) {
     reg_fence32(r);
   } else {
     reg_fence16(r);
@@ -445,17 +467,23 @@ __device__ __forceinline__ void rescale_o_rows(uint32_t tO, float alpha_a, float
 // strides (row, head, batch); otherwise all four are dense [B, H, rows, d] and
 // the maps 3-D (d, rows, B H).
 template <int D, int BN, bool kStrided>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                          const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_o, const Params p) {
   using C = Cfg<D, BN>;
+  using Lay = Layout<BN>;
+  constexpr int kNQ = Lay::kNQ;
+  constexpr int kProducerWarp = Lay::kProducerWarp;
+  constexpr int kMmaWarp = Lay::kMmaWarp;
   extern __shared__ uint8_t smem_raw[];
   // 128-byte-swizzled tiles need 1024-byte-aligned shared-memory addresses
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + C::kSmemQ;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemQ + C::kSmemKV);
+  uint8_t* sO = smem + C::kSmemQ + C::kSmemKV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemQ + C::kSmemKV + C::kSmemO);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -504,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // runs inside the branch that set its register count, so the compiler
   // allocates each role's code under its own limit.
   if (warp >= kProducerWarp) {
-    regs_shrink<kOtherRegs>();
+    regs_shrink<Lay::kOtherRegs>();
     if (warp == kProducerWarp) {
       // ------------------------------------------------------------ producer
       // The whole warp walks the schedule (its counters stay warp-uniform);
@@ -512,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool leader = elect_one_sync();
       {
         int kv_it = 0;
-        int q_cnt[kNQ] = {0, 0};
+        int q_cnt[kNQ] = {};
         bool ok = true;
         for (int k = 0, u = unit_of(0, p); ok && u < p.num_units; u = unit_of(++k, p)) {
           const Unit w = decode_unit<BN>(u, p);
@@ -537,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++q_cnt[t];
             return true;
           };
-          ok = load_q(0) && load_q(1);
+          for (int t = 0; ok && t < kNQ; ++t) ok = load_q(t);
           for (int j = w.ulo; ok && j < w.uhi; ++j) {
   #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
@@ -649,12 +677,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         for (int k = 0, u = unit_of(0, p); ok && u < p.num_units; u = unit_of(++k, p)) {
           // key-block ranges of the two Q tiles (empty range: tile absent)
-          int lo0, hi0, lo1, hi1;
+          int lo0, hi0, lo1 = 0, hi1 = 0;  // a one-tile unit has no tile 1
           {
             const TileWork w0 = decode_tile<BN>(u, 0, p);
-            const TileWork w1 = decode_tile<BN>(u, 1, p);
             lo0 = w0.lo; hi0 = w0.valid ? w0.hi : w0.lo;
-            lo1 = w1.lo; hi1 = w1.valid ? w1.hi : w1.lo;
+            if constexpr (kNQ == 2) {
+              const TileWork w1 = decode_tile<BN>(u, 1, p);
+              lo1 = w1.lo; hi1 = w1.valid ? w1.hi : w1.lo;
+            }
           }
           const bool has0 = hi0 > lo0, has1 = hi1 > lo1;
           const int ulo = has0 ? (has1 ? min(lo0, lo1) : lo0) : (has1 ? lo1 : 0);
@@ -732,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // 32q..32q+15 and 32q+16..32q+31).  Four threads share a row: lane l holds
     // rows l/4 and l/4 + 8 of its warp's 16, and the key columns 8m + 2(l%4)
     // and 8m + 2(l%4) + 1 of every group of eight.
-    regs_grow<kSoftmaxRegs>();
+    regs_grow<Lay::kSoftmaxRegs>();
     const int t = warp / kSoftmaxWarps;
     const int wl = warp % kSoftmaxWarps;
     const int lbase = 32 * (warp % 4) + 16 * (wl / 4);  // first row (= lane) of this warp
@@ -954,27 +984,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(bar(C::kBarOEmpty + t));
       // register 4m + {0, 1}: row a, columns 8m + 2 t0 + {0, 1}; 4m + {2, 3}: row b
       if (p.o_part == nullptr) {
-        size_t off_a, off_b;  // element offsets of the thread's two rows in out
-        if constexpr (kStrided) {
-          const size_t o_head = static_cast<size_t>(w.bh / p.H) * p.o_batch +
-                                static_cast<size_t>(w.bh % p.H) * p.o_head;
-          off_a = o_head + static_cast<size_t>(ok_a ? row_a : 0) * p.o_row;
-          off_b = o_head + static_cast<size_t>(ok_b ? row_b : 0) * p.o_row;
-        } else {
-          off_a = (static_cast<size_t>(w.bh) * p.L + (ok_a ? row_a : 0)) * D;
-          off_b = (static_cast<size_t>(w.bh) * p.L + (ok_b ? row_b : 0)) * D;
-        }
-        uint32_t* dst_a = reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + off_a);
-        uint32_t* dst_b = reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.out) + off_b);
+        // O / l -> bf16 into this warp's 16-row staging box, laid out as the
+        // TMA's 128-byte swizzle (16-byte unit u of row r at u ^ (r % 8)),
+        // then one TMA store per 64-column chunk: coalesced full-line writes,
+        // rows past L clipped by the tensor map.  The lane's rows in the box
+        // are lane / 4 and lane / 4 + 8 (same r % 8), its 4-byte slot 4 t0.
+        uint8_t* box = sO + warp * C::kOBoxBytes;
+        const int r_box = lane / 4;
+        const int warp_row0 = w.q_first + lbase;  // the box's first row in the head
 #pragma unroll
-        for (int m = 0; m < D / 8; ++m) {
-          const int col2 = 4 * m + t0;  // pair index in the row
-          const uint32_t va = pack_bf16x2(__uint_as_float(o[4 * m]) * inv_a,
-                                          __uint_as_float(o[4 * m + 1]) * inv_a);
-          const uint32_t vb = pack_bf16x2(__uint_as_float(o[4 * m + 2]) * inv_b,
-                                          __uint_as_float(o[4 * m + 3]) * inv_b);
-          if (ok_a && in_bounds(off_a + 2 * col2 + 1, p.o_extent)) dst_a[col2] = va;
-          if (ok_b && in_bounds(off_b + 2 * col2 + 1, p.o_extent)) dst_b[col2] = vb;
+        for (int c = 0; c < C::kDChunks; ++c) {
+          if (lane == 0) bulk_wait_group_read0();  // the box's previous store has read it
+          __syncwarp();
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int m = 8 * c + u;  // column group: columns 8m + 2 t0 + {0, 1}
+            const uint32_t va = pack_bf16x2(__uint_as_float(o[4 * m]) * inv_a,
+                                            __uint_as_float(o[4 * m + 1]) * inv_a);
+            const uint32_t vb = pack_bf16x2(__uint_as_float(o[4 * m + 2]) * inv_b,
+                                            __uint_as_float(o[4 * m + 3]) * inv_b);
+            const int slot = ((u ^ (r_box & 7)) * 16) + 4 * t0;
+            *reinterpret_cast<uint32_t*>(box + r_box * 128 + slot) = va;
+            *reinterpret_cast<uint32_t*>(box + (r_box + 8) * 128 + slot) = vb;
+          }
+          fence_proxy_async_shared();
+          __syncwarp();
+          if (lane == 0 && warp_row0 < p.L) {
+            if constexpr (kStrided)
+              tma_store_4d(&tm_o, smem_addr(box), c * 64, warp_row0, w.bh % p.H, w.bh / p.H);
+            else
+              tma_store_3d(&tm_o, smem_addr(box), c * 64, warp_row0, w.bh);
+            bulk_commit_group();
+          }
         }
         if (t0 == 0 && p.lse != nullptr) {
           const size_t n_lse = static_cast<size_t>(p.BH) * p.L;
@@ -1011,6 +1052,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  if (warp < kProducerWarp && lane == 0) bulk_wait_group0();  // epilogue stores complete
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
@@ -1103,6 +1145,7 @@ int launch_t(const FwdArgs& a, cudaStream_t stream, cudaError_t* err) {
   // 0.5-3.5 % faster than the strided instantiation on dense data)
   bool strided = false;
   for (int x = 0; x < 4; ++x) strided = strided || a.stride[x][0] != 0;
+  using Lay = Layout<BN>;
   auto kernel = strided ? attn_fwd_sm100_kernel<D, BN, true> : attn_fwd_sm100_kernel<D, BN, false>;
   int device = 0;
   if ((*err = cudaGetDevice(&device)) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -1122,7 +1165,7 @@ int launch_t(const FwdArgs& a, cudaStream_t stream, cudaError_t* err) {
       // at launch; refuse to launch a build where that does not hold.
       cudaFuncAttributes fa;
       if ((*err = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess) return ATTN_ERR_CUDA;
-      if (fa.numRegs != kLaunchRegs) {
+      if (fa.numRegs != Lay::kLaunchRegs) {
         *err = cudaErrorInvalidConfiguration;
         return ATTN_ERR_CUDA;
       }
@@ -1143,8 +1186,10 @@ int launch_t(const FwdArgs& a, cudaStream_t stream, cudaError_t* err) {
     st[x][1] = dense ? rows * D : a.stride[x][1];
     st[x][2] = dense ? static_cast<long long>(a.H) * rows * D : a.stride[x][2];
   }
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_map(&tq, a.q, a.B, a.H, a.L, D, st[0], kBM, strided, err)) return ATTN_ERR_CUDA;
+  // output: 16-row boxes, one per softmax warp's epilogue store
+  if (!make_map(&to, a.out, a.B, a.H, a.L, D, st[3], 16, strided, err)) return ATTN_ERR_CUDA;
   if (!make_map(&tk, a.k, a.B, a.H, Lk, D, st[1], BN, strided, err)) return ATTN_ERR_CUDA;
   if (!make_map(&tv, a.v, a.B, a.H, Lk, D, st[2], BN, strided, err)) return ATTN_ERR_CUDA;
 
@@ -1164,7 +1209,7 @@ int launch_t(const FwdArgs& a, cudaStream_t stream, cudaError_t* err) {
   p.mask_kind = a.mask_kind;
   p.window = a.window;
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  p.nqp = (a.L + kUnitRows - 1) / kUnitRows;
+  p.nqp = (a.L + Lay::kUnitRows - 1) / Lay::kUnitRows;
   p.num_splits = 1;
   p.split_blocks = 0;
   p.o_part = nullptr;
@@ -1183,7 +1228,7 @@ int launch_t(const FwdArgs& a, cudaStream_t stream, cudaError_t* err) {
   p.num_units = static_cast<int>(units);
   p.timeout_ns = a.timeout_ns;
   const int grid = p.num_units < nsm ? p.num_units : nsm;
-  kernel<<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  kernel<<<grid, Lay::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, p);
   *err = cudaGetLastError();
   return *err == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
@@ -1194,8 +1239,10 @@ int launch_fwd_bf16_sm100(const FwdArgs& a, cudaStream_t stream, cudaError_t* er
   *err = cudaSuccess;
   if (a.d == 128 && a.block_n == 128) return launch_t<128, 128>(a, stream, err);
   if (a.d == 128 && a.block_n == 64) return launch_t<128, 64>(a, stream, err);
+  if (a.d == 128 && a.block_n == 256) return launch_t<128, 256>(a, stream, err);
   if (a.d == 64 && a.block_n == 128) return launch_t<64, 128>(a, stream, err);
   if (a.d == 64 && a.block_n == 64) return launch_t<64, 64>(a, stream, err);
+  if (a.d == 64 && a.block_n == 256) return launch_t<64, 256>(a, stream, err);
   return ATTN_ERR_UNSUPPORTED;
 }
 
@@ -1222,6 +1269,10 @@ int read_device_status(int device, int reset, cudaError_t* err) {
 }
 
 }  // namespace ebh
+
+// The backward's tensor-core kernels share this translation unit's helpers and
+// its device status word.
+#include "attn_bwd_sm100.cuh"
 
 #ifdef EBH_BOUNDS_CHECK
 // Bounds-checking builds only: the number of refused out-of-range stores

@@ -82,8 +82,12 @@ struct BwdArgs {
   int B, H, L, d;
   float scale;
   int mask_kind, window;
+  uint64_t timeout_ns = 10ull * 1000 * 1000 * 1000;  // limit on each wait (tensor-core path)
 };
 int launch_bwd(const BwdArgs& a, cudaStream_t stream, cudaError_t* err);
+// dQ, dK, dV on the tensor cores (bf16, d in {64, 128}); a.D must already
+// hold the row dots <dO_i, O_i>.  Defined with the forward kernel.
+int launch_bwd_sm100(const BwdArgs& a, cudaStream_t stream, cudaError_t* err);
 
 // The multi-head attention layer (validated).
 struct MhaArgs {

@@ -123,7 +123,12 @@ typedef struct attn_params {
   int mask_kind;
   int window;
   int block_n;            /* keys per block on the bf16 path: 0 (auto = 128),
-                             64 or 128; must be 0 on the fp32 path */
+                             64, 128 or 256; must be 0 on the fp32 path.
+                             64 and 128 run two 128-row query tiles per
+                             work unit (their softmax overlaps the other
+                             tile's products); 256 runs one query tile per
+                             unit (S of 256 columns and O of d columns fill
+                             the tensor memory), with no such overlap */
   uint64_t wait_timeout_ns; /* limit on each wait inside the kernel; 0 = 10 s */
 } attn_params;
 

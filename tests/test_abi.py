@@ -87,7 +87,8 @@ BAD = [
     ("mask -1", dict(mask_kind=-1), ebh.ATTN_ERR_INVALID),
     ("window<0", dict(mask_kind=2, window=-1), ebh.ATTN_ERR_INVALID),
     ("block_n 96", dict(block_n=96), ebh.ATTN_ERR_INVALID),
-    ("block_n 256", dict(block_n=256), ebh.ATTN_ERR_INVALID),
+    ("block_n 512", dict(block_n=512), ebh.ATTN_ERR_INVALID),
+    ("block_n 192", dict(block_n=192), ebh.ATTN_ERR_INVALID),
     ("f32 block_n", dict(dtype=1, block_n=64), ebh.ATTN_ERR_INVALID),
     ("dtype 7", dict(dtype=7), ebh.ATTN_ERR_INVALID),
     ("out aliases q", dict(out=1 << 20), ebh.ATTN_ERR_INVALID),

@@ -48,7 +48,7 @@ def test_forward_stores_stay_in_bounds(debug_library, shape):
     q, k, v = G.rand_qkv(B, H, L, d, seed=L + d)
     for mask, window in (("none", 0), ("causal", 0), ("window", 70), ("causal_window", 90)):
         ref_o, ref_l = G.oracle_full(q, k, v, mask=mask, window=window)
-        for bn in (64, 128):
+        for bn in (64, 128, 256):
             out, lse = G.gpu_forward(q, k, v, mask=mask, window=window, block_n=bn)
             G.check_bf16(out, lse, ref_o, ref_l, f"debug {shape} {mask} bn={bn}")
             _no_violations(debug_library)

@@ -39,13 +39,21 @@ def _oracle(q, k, v, g, mask, window, scale=None):
 
 
 CASES = [
-    # (B, H, L, d, mask, window)
+    # (B, H, L, d, mask, window): ragged and whole tiles, every mask, both
+    # head dims of the tensor-core path
     (1, 2, 300, 64, "none", 0),
     (1, 2, 257, 128, "causal", 0),
     (2, 1, 400, 64, "window", 37),
     (1, 3, 333, 128, "causal_window", 50),
     (1, 1, 1, 64, "causal", 0),
     (1, 2, 1000, 128, "causal", 0),
+    (1, 1, 128, 128, "none", 0),
+    (1, 2, 129, 64, "causal", 0),
+    (2, 2, 777, 128, "window", 200),
+    (1, 2, 513, 64, "causal_window", 0),
+    (1, 1, 640, 128, "window", 0),
+    (3, 5, 250, 64, "causal", 0),
+    (1, 4, 4096, 128, "causal", 0),
 ]
 
 
@@ -87,3 +95,16 @@ def test_backward_invariants_on_gpu():
     dq, dk, dv = _run(q, k, v, g, "causal", 0)
     assert np.abs(dk.sum(axis=2)).max() <= 1e-3
     assert np.abs(dv.sum(axis=2) - g.double().numpy().sum(axis=2)).max() <= 1e-3
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_bf16_backward_invariants(d):
+    """The tensor-core path on bf16 inputs: sum_j dV_j = sum_i dO_i, because
+    every row of P sums to one (up to the bf16 roundings of P and the
+    forward's LSE)."""
+    B, H, L = 1, 2, 700
+    q, k, v = G.rand_qkv(B, H, L, d, seed=21 + d)
+    g = G.rand_qkv(B, H, L, d, seed=22 + d)[0]
+    dq, dk, dv = _run(q, k, v, g, "causal", 0)
+    gs = g.double().numpy().sum(axis=2)
+    assert np.abs(dv.sum(axis=2) - gs).max() <= 2e-2 * np.abs(gs).max()

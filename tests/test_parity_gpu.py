@@ -58,7 +58,7 @@ def test_bf16_small_all_rows(shape, mask, window):
     B, H, L, d = shape
     q, k, v = G.rand_qkv(B, H, L, d, seed=L * 7 + d + window)
     ref_o, ref_l = G.oracle_full(q, k, v, mask=mask, window=window)
-    for bn in (64, 128):
+    for bn in (64, 128, 256):
         out, lse = G.gpu_forward(q, k, v, mask=mask, window=window, block_n=bn)
         G.check_bf16(out, lse, ref_o, ref_l, f"{shape} {mask}{window} bn={bn}")
 
@@ -67,18 +67,20 @@ def test_bf16_small_all_rows(shape, mask, window):
 def test_bf16_scale_argument(d):
     q, k, v = G.rand_qkv(1, 2, 300, d, seed=3)
     for scale in (0.01, 0.3, 1.0):
-        out, lse = G.gpu_forward(q, k, v, mask="causal", scale=scale)
         ref_o, ref_l = G.oracle_full(q, k, v, mask="causal", scale=scale)
-        G.check_bf16(out, lse, ref_o, ref_l, f"scale {scale}")
+        for bn in (128, 256):
+            out, lse = G.gpu_forward(q, k, v, mask="causal", scale=scale, block_n=bn)
+            G.check_bf16(out, lse, ref_o, ref_l, f"scale {scale} bn={bn}")
 
 
 def test_bf16_many_heads_persistent_schedule():
     """More work units than SMs, so every CTA walks several units."""
     q, k, v = G.rand_qkv(3, 37, 600, 64, seed=11)
     for mask, window in (("causal", 0), ("window", 100), ("none", 0), ("causal_window", 77)):
-        out, lse = G.gpu_forward(q, k, v, mask=mask, window=window)
         ref_o, ref_l = G.oracle_full(q, k, v, mask=mask, window=window)
-        G.check_bf16(out, lse, ref_o, ref_l, f"many heads {mask}")
+        for bn in (0, 256):
+            out, lse = G.gpu_forward(q, k, v, mask=mask, window=window, block_n=bn)
+            G.check_bf16(out, lse, ref_o, ref_l, f"many heads {mask} bn={bn}")
 
 
 # ---------------------------------------------------------------- full size
@@ -113,7 +115,7 @@ def test_full_mha_L2048_d64_q_times_8_stress():
     assert np.isfinite(out).all() and np.isfinite(lse).all()
 
 
-@pytest.mark.parametrize("block_n", [64, 128])
+@pytest.mark.parametrize("block_n", [64, 128, 256])
 def test_full_causal_L8192_each_block_size(block_n):
     """Every row of the causal L=8192 workload at each key-block size."""
     _all_rows(ebh.WORKLOADS["causal_bf16_L8192_d128"], block_n=block_n)
@@ -124,8 +126,8 @@ def test_full_causal_L8192_block_sizes_agree():
     bf16 tolerances (blockwise attention does not depend on the block size)."""
     w = ebh.WORKLOADS["causal_bf16_L8192_d128"]
     q, k, v = ebh.make_qkv(w)
-    outs = {bn: G.gpu_forward(q, k, v, mask=w.mask, block_n=bn) for bn in (64, 128)}
-    for a, b in ((64, 128),):
+    outs = {bn: G.gpu_forward(q, k, v, mask=w.mask, block_n=bn) for bn in (64, 128, 256)}
+    for a, b in ((64, 128), (64, 256), (128, 256)):
         assert np.abs(outs[a][0] - outs[b][0]).max() <= G.BF16_OUT_ATOL, (a, b)
         assert np.abs(outs[a][1] - outs[b][1]).max() <= G.BF16_LSE_ATOL, (a, b)
 

@@ -58,7 +58,7 @@ def test_forward_rows_bf16_matches_oracle(case):
     q_all, k, v = G.rand_qkv(B, H, Lk, d, seed=Lk + off)
     q = q_all[:, :, off:off + Lq].contiguous()
     ref_o, ref_l = _rows_reference(q, k, v, off, mask, window)
-    for bn in (64, 128):
+    for bn in (64, 128, 256):
         out, lse = ebh.forward_rows(q.cuda(), k.cuda(), v.cuda(), off, mask=mask, window=window,
                                     block_n=bn)
         torch.cuda.synchronize()

@@ -50,7 +50,7 @@ CASES = [
 def test_splitkv_matches_oracle(shape, mask, window, splits):
     q, k, v = G.rand_qkv(*shape, seed=sum(shape) + splits)
     ref_o, ref_l = G.oracle_full(q, k, v, mask=mask, window=window)
-    for bn in (64, 128):
+    for bn in (64, 128, 256):
         out, lse = _splitkv(q, k, v, splits, mask, window, bn)
         G.check_bf16(out, lse, ref_o, ref_l, f"splitkv {shape} {mask} S={splits} bn={bn}")
 

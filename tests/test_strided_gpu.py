@@ -29,11 +29,14 @@ def test_bshd_layout_matches_oracle(shape, mask, window):
     q, k, v = G.rand_qkv(B, H, L, d, seed=L + d)  # [B, H, L, d]
     ref_o, ref_l = G.oracle_full(q, k, v, mask=mask, window=window)
     to_bshd = lambda t: t.transpose(1, 2).contiguous().cuda()  # noqa: E731
-    out, lse = ebh.forward_bshd(to_bshd(q), to_bshd(k), to_bshd(v), mask=mask, window=window)
-    torch.cuda.synchronize()
-    assert ebh.device_status(0) == ebh.ATTN_OK
-    got = out.transpose(1, 2).double().cpu().numpy()
-    G.check_bf16(got, lse.double().cpu().numpy(), ref_o, ref_l, f"bshd {shape} {mask}")
+    for bn in (0, 256):
+        out, lse = ebh.forward_bshd(to_bshd(q), to_bshd(k), to_bshd(v), mask=mask,
+                                    window=window, block_n=bn)
+        torch.cuda.synchronize()
+        assert ebh.device_status(0) == ebh.ATTN_OK
+        got = out.transpose(1, 2).double().cpu().numpy()
+        G.check_bf16(got, lse.double().cpu().numpy(), ref_o, ref_l,
+                     f"bshd {shape} {mask} bn={bn}")
 
 
 def test_padded_rows_and_swapped_head_batch_order():
