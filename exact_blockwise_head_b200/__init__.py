@@ -40,7 +40,7 @@ EXPORTED = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ex", "attn_strerror", "attn_la
             "attn_fwd_splitkv", "attn_merge", "attn_abi_version", "attn_fwd_splitkv_noalloc",
             "attn_fwd_rows", "attn_seq_unshard", "attn_mha_workspace_bytes", "attn_mha_fwd",
             "attn_bwd_workspace_bytes", "attn_bwd", "attn_query_rows_for_keys",
-            "attn_fwd_strided")
+            "attn_fwd_strided", "attn_fwd_partial", "attn_merge_rows")
 
 
 class AttnParams(ctypes.Structure):
@@ -136,6 +136,9 @@ def _load():
             lib.attn_mha_fwd.argtypes = [ctypes.POINTER(MhaParams), vp, ctypes.c_size_t, vp]
             lib.attn_merge.argtypes = [vp, vp, i, ctypes.POINTER(i), i, i, vp, vp, i, i, i, i, i,
                                        vp]
+            lib.attn_merge_rows.argtypes = [vp, vp, i, ctypes.POINTER(i), i, i, vp, vp, i, i, i, i,
+                                            i, i, i, vp]
+            lib.attn_fwd_partial.argtypes = [ctypes.POINTER(AttnParams), i, i, vp, vp, vp]
             for name in EXPORTED:
                 if name != "attn_strerror":
                     getattr(lib, name).restype = ctypes.c_int
@@ -504,6 +507,75 @@ def merge(o_parts, lse_parts, split_bounds, mask="none", window=0, out_dtype=Non
     if st != ATTN_OK:
         raise AttnError(st, "attn_merge")
     return out, lse
+
+
+def merge_rows(o_parts, lse_parts, split_bounds, kv_len, q_offset, mask="none", window=0,
+               out_dtype=None, out=None, lse=None, stream=None):
+    """merge() for rows at key positions q_offset .. q_offset + L - 1 among
+    kv_len keys (see attn_merge_rows in include/attn.h).  o_parts: fp32
+    [S,B,H,L,d] CUDA; lse_parts: fp32 [S,B,H,L]; split_bounds: S+1 key
+    positions from 0 to kv_len."""
+    import torch
+
+    S, B, H, L, d = o_parts.shape
+    if out_dtype is None:
+        out_dtype = torch.bfloat16
+    if out is None:
+        out = torch.empty((B, H, L, d), dtype=out_dtype, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=o_parts.device)
+    bounds = (ctypes.c_int * (S + 1))(*[int(b) for b in split_bounds])
+    dt = ATTN_DTYPE_BF16 if out.dtype == torch.bfloat16 else ATTN_DTYPE_F32
+    with torch.cuda.device(o_parts.device):
+        st = _load().attn_merge_rows(o_parts.data_ptr(), lse_parts.data_ptr(), S, bounds,
+                                     MASK_KINDS[mask], int(window), out.data_ptr(),
+                                     lse.data_ptr(), dt, B, H, L, d, int(kv_len), int(q_offset),
+                                     _stream_handle(stream, o_parts.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_merge_rows")
+    return out, lse
+
+
+def forward_partial(q, k, v, q_shift, o_part, lse_part, scale=None, mask="none", window=0,
+                    block_n=0, stream=None):
+    """Partial forward of q's rows against one block of keys (see
+    attn_fwd_partial in include/attn.h): query row i sits at key position
+    q_shift + i relative to k's first row (q_shift may be negative).  Writes
+    o_part (fp32 [B, H, L, d]) and lse_part (fp32 [B, H, L]) in place."""
+    import torch
+
+    if q.dim() != 4 or k.shape != v.shape or q.shape[:2] != k.shape[:2] or q.shape[3] != k.shape[3]:
+        raise ValueError("q must be [B, H, L, d] and k, v [B, H, Lk, d]")
+    if not (q.dtype == k.dtype == v.dtype == torch.bfloat16):
+        raise TypeError("q, k, v must be bf16")
+    for name, t in (("q", q), ("k", k), ("v", v), ("o_part", o_part), ("lse_part", lse_part)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    B, H, L, d = q.shape
+    if o_part.shape != (B, H, L, d) or lse_part.shape != (B, H, L) or \
+            o_part.dtype != torch.float32 or lse_part.dtype != torch.float32:
+        raise ValueError("o_part must be fp32 [B, H, L, d] and lse_part fp32 [B, H, L]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if mask not in MASK_KINDS:
+        raise ValueError(f"mask must be one of {sorted(MASK_KINDS)}")
+    p = AttnParams()
+    p.dtype = ATTN_DTYPE_BF16
+    p.q, p.k, p.v = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    p.out, p.lse = o_part.data_ptr(), None
+    p.B, p.H, p.L, p.d = B, H, L, d
+    p.scale = float(scale)
+    p.mask_kind = MASK_KINDS[mask]
+    p.window = int(window)
+    p.block_n = int(block_n)
+    p.wait_timeout_ns = 0
+    with torch.cuda.device(q.device):
+        st = _load().attn_fwd_partial(ctypes.byref(p), int(k.shape[2]), int(q_shift),
+                                      o_part.data_ptr(), lse_part.data_ptr(),
+                                      _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_partial")
+    return o_part, lse_part
 
 
 def device_status(device: int = 0, reset: bool = True) -> int:

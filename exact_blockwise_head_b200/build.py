@@ -5,8 +5,8 @@
 The library is the C ABI of include/attn.h: api.cpp (validation, dispatch),
 attn_sm100.cu (tcgen05 bf16 kernel), attn_f32.cu (fp32 CUDA-core kernel), the
 split-KV merge, sequence-shard layout, multi-head layer and backward kernels.
-The CUDA runtime is linked statically; cuBLASLt (the layer's projections) is
-linked dynamically.  Two variants build beside it: libebh_attn_trace.so
+The CUDA runtime is linked statically; no other CUDA library is linked (the
+layer's projections run in the library's own tensor-core GEMM).  Two variants build beside it: libebh_attn_trace.so
 (pipeline timestamps) and libebh_attn_debug.so (bounds-checked stores).
 """
 from __future__ import annotations
@@ -24,7 +24,7 @@ TRACE_LIB = os.path.join(PKG, "libebh_attn_trace.so")
 DEBUG_LIB = os.path.join(PKG, "libebh_attn_debug.so")
 SOURCES = ["api.cpp", "attn_sm100.cu", "attn_f32.cu", "attn_merge.cu", "noalloc.cu",
            "seqpar.cu", "mha.cu", "attn_bwd.cu"]
-HEADERS = ["kernels.h", "sm100_ptx.cuh", "tiles.h", "attn_bwd_sm100.cuh"]
+HEADERS = ["kernels.h", "sm100_ptx.cuh", "tiles.h", "attn_bwd_sm100.cuh", "linear_sm100.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -76,7 +76,6 @@ def build(force: bool = False, verbose: bool = False, trace: bool = False,
     if verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
-    cmd += ["-lcublasLt"]  # the layer's two projections
     subprocess.run(cmd, check=True)
     os.replace(tmp, target)
     return target

@@ -353,9 +353,9 @@ int attn_mha_fwd(const attn_mha_params* p, void* workspace, size_t workspace_byt
   a.window = has_window(p->mask_kind) ? (p->window > p->L ? p->L : p->window) : 0;
   a.timeout_ns = kDefaultTimeoutNs;
   cudaError_t err = cudaSuccess;
-  int lt = 0;
-  st = ebh::launch_mha(a, workspace, static_cast<cudaStream_t>(stream), &err, &lt);
-  if (st == ATTN_ERR_CUDA) g_last_cuda_error = lt != 0 ? -lt : static_cast<int>(err);
+  int proj = 0;
+  st = ebh::launch_mha(a, workspace, static_cast<cudaStream_t>(stream), &err, &proj);
+  if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
   return st;
 }
 
@@ -507,18 +507,22 @@ int attn_fwd_splitkv(const attn_params* p, int num_splits, void* workspace,
   m.d = a.d;
   m.mask_kind = a.mask_kind;
   m.window = a.window;
+  m.kv_len = a.L;
+  m.q_offset = 0;
   st = ebh::launch_merge(m, static_cast<cudaStream_t>(stream), &err);
   if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
   return st;
 }
 
-int attn_merge(const float* o_parts, const float* lse_parts, int num_splits,
-               const int* split_bounds, int mask_kind, int window, void* out, float* lse,
-               int out_dtype, int B, int H, int L, int d, void* stream) {
+int attn_merge_rows(const float* o_parts, const float* lse_parts, int num_splits,
+                    const int* split_bounds, int mask_kind, int window, void* out, float* lse,
+                    int out_dtype, int B, int H, int L, int d, int kv_len, int q_offset,
+                    void* stream) {
   if (!o_parts || !lse_parts || !split_bounds || !out) return ATTN_ERR_INVALID;
   if (num_splits < 1 || num_splits > ebh::kMaxSplits) return ATTN_ERR_INVALID;
-  if (B <= 0 || H <= 0 || L <= 0) return ATTN_ERR_INVALID;
+  if (B <= 0 || H <= 0 || L <= 0 || kv_len <= 0) return ATTN_ERR_INVALID;
   if (static_cast<long long>(B) * H > 0x7fffffffLL) return ATTN_ERR_INVALID;
+  if (q_offset < 0 || static_cast<long long>(q_offset) + L > kv_len) return ATTN_ERR_INVALID;
   if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_CAUSAL_WINDOW) return ATTN_ERR_INVALID;
   if (has_window(mask_kind) && window < 0) return ATTN_ERR_INVALID;
   if (out_dtype != ATTN_DTYPE_BF16 && out_dtype != ATTN_DTYPE_F32) return ATTN_ERR_INVALID;
@@ -526,7 +530,7 @@ int attn_merge(const float* o_parts, const float* lse_parts, int num_splits,
   if (split_bounds[0] != 0) return ATTN_ERR_INVALID;
   for (int s = 0; s < num_splits; ++s)
     if (split_bounds[s + 1] < split_bounds[s]) return ATTN_ERR_INVALID;
-  if (split_bounds[num_splits] != L) return ATTN_ERR_INVALID;
+  if (split_bounds[num_splits] != kv_len) return ATTN_ERR_INVALID;
   if (!aligned(o_parts, 16) || !aligned(lse_parts, 4) || !aligned(out, 16) ||
       (lse && !aligned(lse, 4)))
     return ATTN_ERR_MISALIGNED;
@@ -544,9 +548,64 @@ int attn_merge(const float* o_parts, const float* lse_parts, int num_splits,
   m.L = L;
   m.d = d;
   m.mask_kind = mask_kind;
-  m.window = has_window(mask_kind) ? (window > L ? L : window) : 0;
+  m.window = has_window(mask_kind) ? (window > kv_len ? kv_len : window) : 0;
+  m.kv_len = kv_len;
+  m.q_offset = q_offset;
   cudaError_t err = cudaSuccess;
   st = ebh::launch_merge(m, static_cast<cudaStream_t>(stream), &err);
+  if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
+  return st;
+}
+
+int attn_merge(const float* o_parts, const float* lse_parts, int num_splits,
+               const int* split_bounds, int mask_kind, int window, void* out, float* lse,
+               int out_dtype, int B, int H, int L, int d, void* stream) {
+  return attn_merge_rows(o_parts, lse_parts, num_splits, split_bounds, mask_kind, window, out, lse,
+                         out_dtype, B, H, L, d, L, 0, stream);
+}
+
+int attn_fwd_partial(const attn_params* p, int kv_len, int q_shift, float* o_part,
+                     float* lse_part, void* stream) {
+  if (p == nullptr || o_part == nullptr || lse_part == nullptr) return ATTN_ERR_INVALID;
+  if (p->dtype != ATTN_DTYPE_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (kv_len <= 0) return ATTN_ERR_INVALID;
+  // every key position a row could reach stays inside int: |shift| + L + kv_len
+  const long long reach = (q_shift < 0 ? -static_cast<long long>(q_shift) : q_shift) +
+                          static_cast<long long>(p->L) + kv_len;
+  if (reach > 0x3fffffffLL) return ATTN_ERR_INVALID;
+  // p->out and p->lse are not used: the results go to o_part and lse_part
+  attn_params pc = *p;
+  pc.out = o_part;
+  pc.lse = nullptr;
+  ebh::FwdArgs a;
+  int st = validate(&pc, &a);
+  if (st != ATTN_OK) return st;
+  {  // k and v hold kv_len rows; the partials must not overlap anything
+    const uint64_t rows = static_cast<uint64_t>(p->B) * p->H * p->L;
+    const uint64_t kv_bytes = static_cast<uint64_t>(p->B) * p->H * kv_len * p->d * 2;
+    const uint64_t o_bytes = rows * p->d * 4, l_bytes = rows * 4;
+    const uint64_t q_bytes = rows * p->d * 2;
+    if (!aligned(o_part, 16) || !aligned(lse_part, 4)) return ATTN_ERR_MISALIGNED;
+    const void* ins[3] = {p->q, p->k, p->v};
+    const uint64_t in_sz[3] = {q_bytes, kv_bytes, kv_bytes};
+    for (int x = 0; x < 3; ++x)
+      if (overlap(o_part, o_bytes, ins[x], in_sz[x]) || overlap(lse_part, l_bytes, ins[x], in_sz[x]))
+        return ATTN_ERR_INVALID;
+    if (overlap(o_part, o_bytes, lse_part, l_bytes)) return ATTN_ERR_INVALID;
+  }
+  a.Lk = kv_len;
+  a.q_shift = q_shift;
+  // a band wider than any distance between a row and a key allows every pair
+  a.window = has_window(p->mask_kind) ? static_cast<int>(p->window > reach ? reach : p->window)
+                                      : 0;
+  const int nkv = (kv_len + a.block_n - 1) / a.block_n;
+  a.num_splits = 1;  // one run over all of the given keys, written as a partial
+  a.split_keys = nkv * a.block_n;
+  a.o_part = o_part;
+  a.lse_part = lse_part;
+  if ((st = check_device_sm100()) != ATTN_OK) return st;
+  cudaError_t err = cudaSuccess;
+  st = ebh::launch_fwd_bf16_sm100(a, static_cast<cudaStream_t>(stream), &err);
   if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
   return st;
 }

@@ -621,7 +621,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
-template <int D, typename Kernel>
+// One-time set-up per (kernel, device): the shared-memory limit and the
+// register check.  kWhich tells the two kernels apart (their function types
+// are the same, so the kernel's type alone would share one flag between them).
+template <int D, int kWhich, typename Kernel>
 int bwd_prepare(Kernel kernel, cudaError_t* err) {
   int device = 0;
   if ((*err = cudaGetDevice(&device)) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -649,9 +652,9 @@ int bwd_prepare(Kernel kernel, cudaError_t* err) {
 
 template <int D>
 int launch_bwd_sm100_t(const BwdArgs& a, cudaStream_t stream, cudaError_t* err) {
-  int st = bwd_prepare<D>(bwd_dkdv_sm100_kernel<D>, err);
+  int st = bwd_prepare<D, 0>(bwd_dkdv_sm100_kernel<D>, err);
   if (st != ATTN_OK) return st;
-  if ((st = bwd_prepare<D>(bwd_dq_sm100_kernel<D>, err)) != ATTN_OK) return st;
+  if ((st = bwd_prepare<D, 1>(bwd_dq_sm100_kernel<D>, err)) != ATTN_OK) return st;
   const int BH = a.B * a.H;
   const long long dense[3] = {D, static_cast<long long>(a.L) * D,
                               static_cast<long long>(a.H) * a.L * D};

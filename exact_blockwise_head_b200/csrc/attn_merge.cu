@@ -7,7 +7,8 @@
 // the combination step the page "Mosaic multi-GPU sequence-sharded attention"
 // (kwkr.cn), section 2.1, calls the tree reduction of local attention results.
 // Splits whose key range holds no allowed key of a row are skipped for that
-// row (they were never written for it).  One warp per row; each lane owns
+// row (they were never written for it).  Rows may sit at an offset into the
+// keys (a rank's rows of a sequence-sharded problem).  One warp per row; each lane owns
 // d/32 consecutive columns, read as one vector.
 #include <cuda_runtime.h>
 
@@ -32,16 +33,17 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Merg
   const int bh = static_cast<int>(row / m.L);
   const int i = static_cast<int>(row % m.L);
 
-  // allowed keys of row i: [kmin, kmax]
-  long long kmin = 0, kmax = m.L - 1;
+  // allowed keys of row i (key position qp): [kmin, kmax]
+  const long long qp = static_cast<long long>(m.q_offset) + i;
+  long long kmin = 0, kmax = static_cast<long long>(m.kv_len) - 1;
   if (m.mask_kind == kMaskCausal) {
-    kmax = i;
+    kmax = qp < kmax ? qp : kmax;
   } else if (m.mask_kind == kMaskWindow) {
-    kmin = (long long)i - m.window > 0 ? (long long)i - m.window : 0;
-    kmax = (long long)i + m.window < m.L - 1 ? (long long)i + m.window : m.L - 1;
+    kmin = qp - m.window > 0 ? qp - m.window : 0;
+    kmax = qp + m.window < kmax ? qp + m.window : kmax;
   } else if (m.mask_kind == kMaskCausalWindow) {
-    kmin = (long long)i - m.window > 0 ? (long long)i - m.window : 0;
-    kmax = i;
+    kmin = qp - m.window > 0 ? qp - m.window : 0;
+    kmax = qp < kmax ? qp : kmax;
   }
   auto contributes = [&](int s) {
     const long long lo = m.bounds[s] > kmin ? m.bounds[s] : kmin;

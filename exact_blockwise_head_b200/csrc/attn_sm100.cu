@@ -47,8 +47,6 @@ namespace ebh {
 namespace {
 
 constexpr int kBM = 128;          // query rows per Q tile (= tensor-memory lanes)
-constexpr int kSoftmaxWarps = 8;   // per Q tile: two per tensor-memory sub-partition
-constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
 
 // Work-unit shape per key-block size.  With 64- and 128-key blocks a unit is
 // two 128-row Q tiles that share the K/V stream (S_0 | S_1 | O_0 | O_1 fill
@@ -57,6 +55,10 @@ constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
 template <int BN>
 struct Layout {
   static constexpr int kNQ = BN == 256 ? 1 : 2;  // Q tiles per work unit
+  // softmax warps per Q tile: two per tensor-memory sub-partition, four
+  // threads per row (16-lane shapes)
+  static constexpr int kSoftmaxWarps = 8;
+  static constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
   static constexpr int kUnitRows = kBM * kNQ;
   static constexpr int kThreads = (kNQ * kSoftmaxWarps + 4) * 32;  // + producer, MMA, 2 idle
   static constexpr int kProducerWarp = kNQ * kSoftmaxWarps;
@@ -66,6 +68,8 @@ struct Layout {
   // softmax: a BN/2-wide half row block per thread plus its packed bf16 copy
   static constexpr int kSoftmaxRegs = kNQ == 2 ? 104 : 208;
   static constexpr int kOtherRegs = 64;
+  // epilogue staging rows per softmax warp (its rows of the Q tile)
+  static constexpr int kOBoxRows = 16;
   static_assert(kSoftmaxRegs * kNQ * kSoftmaxThreads + kOtherRegs * 128 <=
                     kLaunchRegs * kThreads,
                 "register split exceeds the launch allocation");
@@ -148,8 +152,8 @@ struct Cfg {
   static constexpr int kSmemKV = kStages * kKVTileBytes;
   // epilogue staging: one 16-row x 64-column bf16 box (128-byte swizzle) per
   // softmax warp, written by the warp and stored by TMA
-  static constexpr int kOBoxBytes = 16 * 128;
-  static constexpr int kSmemO = kNQ * kSoftmaxWarps * kOBoxBytes;
+  static constexpr int kOBoxBytes = Layout<BN>::kOBoxRows * 128;
+  static constexpr int kSmemO = kNQ * Layout<BN>::kSoftmaxWarps * kOBoxBytes;
   // barrier indices
   static constexpr int kBarQFull = 0;                  // [kNQ]
   static constexpr int kBarQEmpty = kBarQFull + kNQ;   // [kNQ]
@@ -226,7 +230,13 @@ __device__ __forceinline__ TileWork decode_tile(int u, int t, const Params& p) {
   if (w.valid) {
     kv_tile_range(p.Lk, w.q_first + p.q_shift, w.q_last + p.q_shift, p.mask_kind, p.window, BN,
                   w.lo, w.hi);
-    if (p.num_splits > 1) {
+    if (w.hi <= w.lo) {
+      // no key block to visit (query rows placed outside a key shard's
+      // reach): the tile does no work and writes nothing
+      w.valid = false;
+      w.lo = w.hi = 0;
+    }
+    if (w.valid && p.num_splits > 1) {
       w.lo = max(w.lo, w.split * p.split_blocks);
       w.hi = min(w.hi, (w.split + 1) * p.split_blocks);
       if (w.hi <= w.lo) {
@@ -477,6 +487,8 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
   constexpr int kNQ = Lay::kNQ;
   constexpr int kProducerWarp = Lay::kProducerWarp;
   constexpr int kMmaWarp = Lay::kMmaWarp;
+  constexpr int kSoftmaxWarps = Lay::kSoftmaxWarps;
+  constexpr int kSoftmaxThreads = Lay::kSoftmaxThreads;
   extern __shared__ uint8_t smem_raw[];
   // 128-byte-swizzled tiles need 1024-byte-aligned shared-memory addresses
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
@@ -1052,7 +1064,9 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
     }
   }
 
-  if (warp < kProducerWarp && lane == 0) bulk_wait_group0();  // epilogue stores complete
+  // the epilogue's staging boxes must have been read before the CTA's shared
+  // memory goes; the global writes complete with the kernel
+  if (warp < kProducerWarp && lane == 0) bulk_wait_group_read0();
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
@@ -1189,7 +1203,8 @@ int launch_t(const FwdArgs& a, cudaStream_t stream, cudaError_t* err) {
   CUtensorMap tq, tk, tv, to;
   if (!make_map(&tq, a.q, a.B, a.H, a.L, D, st[0], kBM, strided, err)) return ATTN_ERR_CUDA;
   // output: 16-row boxes, one per softmax warp's epilogue store
-  if (!make_map(&to, a.out, a.B, a.H, a.L, D, st[3], 16, strided, err)) return ATTN_ERR_CUDA;
+  if (!make_map(&to, a.out, a.B, a.H, a.L, D, st[3], Lay::kOBoxRows, strided, err))
+    return ATTN_ERR_CUDA;
   if (!make_map(&tk, a.k, a.B, a.H, Lk, D, st[1], BN, strided, err)) return ATTN_ERR_CUDA;
   if (!make_map(&tv, a.v, a.B, a.H, Lk, D, st[2], BN, strided, err)) return ATTN_ERR_CUDA;
 
@@ -1273,6 +1288,7 @@ int read_device_status(int device, int reset, cudaError_t* err) {
 // The backward's tensor-core kernels share this translation unit's helpers and
 // its device status word.
 #include "attn_bwd_sm100.cuh"
+#include "linear_sm100.cuh"
 
 #ifdef EBH_BOUNDS_CHECK
 // Bounds-checking builds only: the number of refused out-of-range stores

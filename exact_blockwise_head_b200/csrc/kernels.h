@@ -47,12 +47,16 @@ struct MergeArgs {
   const float* o_part;
   const float* lse_part;
   int num_splits;
-  int bounds[kMaxSplits + 1];
+  int bounds[kMaxSplits + 1];  // key positions, from 0 to kv_len
   void* out;           // bf16 or fp32 [B,H,L,d]
   float* lse;          // fp32 [B,H,L] or nullptr
   bool out_f32;
   int BH, L, d;
   int mask_kind, window;
+  // row i of the L rows sits at key position q_offset + i among kv_len keys
+  // (0 and L for a plain split-KV merge)
+  int kv_len = 0;
+  int q_offset = 0;
 };
 
 // Each returns an ATTN_* status; on ATTN_ERR_CUDA *err holds the CUDA code.
@@ -103,9 +107,15 @@ struct MhaArgs {
   uint64_t timeout_ns;
 };
 size_t mha_workspace_bytes(int B, int L, int E);
-// On ATTN_ERR_CUDA, *err holds a CUDA error or *lt_status a cuBLASLt failure.
+// Y[M, N] = X[M, K] W[N, K]^T + bias[N] (bias may be null), bf16 in and out,
+// fp32 accumulation, on the tensor cores; N and K multiples of 8.  Defined
+// with the attention kernels.
+int launch_linear_bf16(const void* x, const void* w, const void* bias, void* y, int M, int N, int K,
+                       uint64_t timeout_ns, cudaStream_t stream, cudaError_t* err);
+// On failure *err holds the CUDA error and *proj the failing projection (1 the
+// qkv projection, 2 the output projection; 0 the attention).
 int launch_mha(const MhaArgs& a, void* workspace, cudaStream_t stream, cudaError_t* err,
-               int* lt_status);
+               int* proj);
 
 // Every argument check of attn_fwd_splitkv except those on the workspace
 // (defined in api.cpp).  On ATTN_OK, *runs is the number of key runs the call

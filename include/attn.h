@@ -252,6 +252,43 @@ ATTN_API int attn_merge(const float* o_parts, const float* lse_parts, int num_sp
                         float* lse, int out_dtype, int B, int H, int L, int d, void* stream);
 
 /*
+ * attn_merge for rows placed inside a longer key sequence: row i of the L
+ * rows sits at key position q_offset + i among kv_len keys, and split_bounds
+ * (S+1 increasing key positions from 0 to kv_len) partition those keys.  A
+ * split is read for a row only when its key range holds a key the row may
+ * attend to.  0 <= q_offset, q_offset + L <= kv_len.  attn_merge is this call
+ * with kv_len = L and q_offset = 0.  This is the combination step of
+ * sequence-sharded attention ("Mosaic multi-GPU sequence-sharded attention",
+ * section 2.1): each rank merges the partials of its rows over every key
+ * shard.  Other arguments and errors as attn_merge.
+ */
+ATTN_API int attn_merge_rows(const float* o_parts, const float* lse_parts, int num_splits,
+                             const int* split_bounds, int mask_kind, int window, void* out,
+                             float* lse, int out_dtype, int B, int H, int L, int d, int kv_len,
+                             int q_offset, void* stream);
+
+/*
+ * Partial forward of query rows against one block of keys, for merging with
+ * attn_merge / attn_merge_rows: q is [B, H, L, d], k and v are [B, H, kv_len,
+ * d] (bf16), and query row i sits at key position q_shift + i relative to
+ * the first of these keys; q_shift may be negative or beyond kv_len (a key
+ * shard that lies after or before the rows), and the masks compare those
+ * positions.  Writes o_part: fp32 [B, H, L, d], the output over these keys
+ * alone (normalised within them), and lse_part: fp32 [B, H, L], its
+ * natural-log LSE.  A row with no allowed key among them gets O = 0 and LSE =
+ * -inf when its 128-row tile has an allowed key for some other row; a tile
+ * with no allowed key at all is not written (the merge's mask rule never
+ * reads it).  p->out and p->lse are not used; p->block_n as attn_fwd_ex.
+ * o_part (16-byte aligned) and lse_part (4-byte aligned) are device memory
+ * and overlap nothing else; |q_shift| + L + kv_len must stay below 2^30.
+ * This is the local step of sequence-sharded attention ("Mosaic multi-GPU
+ * sequence-sharded attention", section 2.1) for one shard of the keys.
+ * Asynchronous on `stream`; allocates nothing.  Errors as attn_fwd_ex.
+ */
+ATTN_API int attn_fwd_partial(const attn_params* p, int kv_len, int q_shift, float* o_part,
+                              float* lse_part, void* stream);
+
+/*
  * Split-KV forward with no workspace argument and no allocation.  The paper
  * has no counterpart to this call: it is a library convenience for callers
  * that cannot allocate device memory for attn_fwd_splitkv's workspace, such
@@ -323,16 +360,16 @@ ATTN_API int attn_bwd(const attn_params* p, const void* dout, float* dq, float* 
  * x, y: bf16 [B, L, E]; w_qkv: bf16 [3E, E] (nn.Linear layout: row j makes
  * output feature j; rows [0, E) make q, [E, 2E) k, [2E, 3E) v); w_out: bf16
  * [E, E]; b_qkv [3E] and b_out [E]: bf16 or NULL.  d in {64, 128}; every
- * pointer 16-byte aligned.  The projections run in cuBLASLt (fp32
- * accumulation, bias in its epilogue, bf16 results); the attention runs in
- * this library's kernel, reading each head's q, k, v straight from the
- * projection output and writing the context in [B, L, H, d] (the head split
- * and merge are its strides).  The projection output and the context are
- * bf16 in `workspace`: device memory, 256-byte aligned, at least
- * attn_mha_workspace_bytes(B, L, E) bytes, disjoint from the other
- * arguments.  On a cuBLASLt failure the call returns ATTN_ERR_CUDA
- * and attn_last_cuda_error() returns -(1 for the first projection, 2 for the
- * second).  Asynchronous on `stream`.
+ * pointer 16-byte aligned.  The projections run in this library's
+ * tensor-core GEMM (tcgen05 MMAs, fp32 accumulation in tensor memory, bias in
+ * its epilogue, bf16 results); the attention runs in this library's kernel,
+ * reading each head's q, k, v straight from the projection output and
+ * writing the context in [B, L, H, d] (the head split and merge are its
+ * strides).  The projection output and the context are bf16 in `workspace`:
+ * device memory, 256-byte aligned, at least attn_mha_workspace_bytes(B, L, E)
+ * bytes, disjoint from the other arguments.  A failed launch returns
+ * ATTN_ERR_CUDA with its code in attn_last_cuda_error().  Asynchronous on
+ * `stream`.
  */
 typedef struct {
   const void* x;

@@ -42,7 +42,13 @@ def test_mha_argument_checks_without_a_device(lib):
     assert lib.attn_mha_fwd(None, None, 0, None) == ebh.ATTN_ERR_INVALID
     assert lib.attn_mha_fwd(ctypes.byref(p), None, 0, None) == ebh.ATTN_ERR_INVALID
     assert lib.attn_mha_workspace_bytes(0, 1, 64) == 0
-    assert lib.attn_mha_workspace_bytes(1, 8, 64) > 8 * 64 * 2 * 8
+    # the bf16 qkv projection output (3 E per row) and the context (E per
+    # row), each rounded up to 256 bytes
+    act = 8 * 64 * 2
+    assert lib.attn_mha_workspace_bytes(1, 8, 64) == -(-3 * act // 256) * 256 + -(-act // 256) * 256
+    act = 3 * 100 * 192 * 2
+    assert lib.attn_mha_workspace_bytes(3, 100, 192) == \
+        -(-3 * act // 256) * 256 + -(-act // 256) * 256
 
 
 def test_abi_version_and_strerror(lib):

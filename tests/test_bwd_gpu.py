@@ -67,7 +67,11 @@ def test_bf16_backward_matches_oracle(case):
     for name, a, b in zip(("dq", "dk", "dv"), got, ref):
         assert np.isfinite(a).all()
         err = np.abs(a - b).max()
-        assert err <= 2e-2 * np.abs(b).max(), f"{case} {name}: {err:.3e} vs max {np.abs(b).max():.3e}"
+        # With window 0 every row attends to its own key only, so dS = 0 and
+        # the exact dQ and dK vanish; the bound then rests on a floor of 1e-3
+        # for the gradient scale (the inputs and dO are O(1)).
+        bound = 2e-2 * max(np.abs(b).max(), 1e-3)
+        assert err <= bound, f"{case} {name}: {err:.3e} vs max {np.abs(b).max():.3e}"
 
 
 @pytest.mark.parametrize("L,d,mask,window", [(200, 40, "causal", 0), (130, 17, "window", 9),

@@ -45,6 +45,10 @@ CASES = [
     (1, 400, 512, 4, "window", 50, False),
     (2, 333, 256, 2, "causal_window", 100, True),
     (2, 512, 512, 8, "causal", 0, True),
+    # E = 192 (3 heads of 64): the projections' N (576, 192) is not a whole
+    # number of 128-column GEMM tiles, and B L = 131 rows leaves a ragged M tile
+    (1, 131, 192, 3, "causal", 0, True),
+    (3, 77, 384, 6, "none", 0, False),
 ]
 
 

@@ -1,11 +1,11 @@
 """Sequence-sharded forward across ranks: the orchestration on CPU gloo ranks.
 
 "Mosaic multi-GPU sequence-sharded attention", section 2.1: rank r holds rows
-[r Ls, (r+1) Ls) of Q, K and V.  These tests run the real gather step (a
-torch.distributed collective, here over gloo) with the other two steps done on
-the CPU: the layout change as an array transpose and the local forward by the
-fp64 oracle on the rank's rows.  The rows every rank returns must be the
-unsharded definition's rows.
+[r Ls, (r+1) Ls) of Q, K and V.  These tests run the real ring exchange (a
+torch.distributed point-to-point batch, here over gloo) with the other steps
+done on the CPU: each shard's partial by the fp64 oracle over that shard's
+keys, the merge in numpy.  The rows every rank returns must be the unsharded
+definition's rows.
 """
 import os
 import socket
@@ -26,24 +26,64 @@ def test_shard_offsets():
 
 
 class _CpuOps(seqpar.DeviceOps):
-    """gather as on the GPUs; unshard and the local forward on the CPU."""
+    """The exchange as on the GPUs (torch.distributed point-to-point, here
+    over gloo); the partial by the fp64 oracle over the shard's key range; the
+    merge in numpy, over the shards a row's partial was computed for."""
 
-    def unshard(self, gathered):
-        S, B, H, Ls, d = gathered.shape
-        return gathered.permute(1, 2, 0, 3, 4).reshape(B, H, S * Ls, d)
-
-    def local(self, q, k_full, v_full, q_offset, scale, mask, window, block_n):
+    def single(self, q, k, v, scale, mask, window, block_n):
         import oracle
 
+        o, l = oracle.attention(q.numpy(), k.numpy(), v.numpy(), scale=scale, mask=mask,
+                                window=window)
+        return o, l
+
+    def parts(self, world, q):
         B, H, Ls, d = q.shape
-        L = k_full.shape[2]
-        q_full = torch.zeros(B, H, L, d)
-        q_full[:, :, q_offset:q_offset + Ls] = q
-        bh = np.repeat(np.arange(B * H), Ls)
-        rows = np.tile(np.arange(q_offset, q_offset + Ls), B * H)
-        o, l = oracle.attention_rows(q_full.numpy(), k_full.numpy(), v_full.numpy(), bh, rows,
-                                     scale=scale, mask=mask, window=window)
-        return o.reshape(B, H, Ls, d), l.reshape(B, H, Ls)
+        return (torch.full((world, B, H, Ls, d), float("nan"), dtype=torch.float64),
+                torch.full((world, B, H, Ls), float("-inf"), dtype=torch.float64))
+
+    def partial(self, q, k, v, q_shift, o_part, lse_part, scale, mask, window, block_n):
+        import oracle
+
+        # rows at key positions q_shift + i, the shard's keys at 0 .. Lk - 1:
+        # place both on one axis starting at min(0, q_shift)
+        B, H, Ls, d = q.shape
+        Lk = k.shape[2]
+        lo = min(0, q_shift)
+        total = max(Lk, q_shift + Ls) - lo
+        qf, kf, vf = (torch.zeros(B, H, total, d) for _ in range(3))
+        qf[:, :, q_shift - lo:q_shift - lo + Ls] = q
+        kf[:, :, -lo:-lo + Lk] = k
+        vf[:, :, -lo:-lo + Lk] = v
+        o, l = oracle.attention_partial(qf.numpy(), kf.numpy(), vf.numpy(), -lo, -lo + Lk,
+                                        scale=scale, mask=mask, window=window)
+        o_part[...] = torch.from_numpy(o[:, :, q_shift - lo:q_shift - lo + Ls])
+        lse_part[...] = torch.from_numpy(l[:, :, q_shift - lo:q_shift - lo + Ls])
+
+    def merge(self, o_parts, lse_parts, bounds, kv_len, q_offset, mask, window, out_dtype):
+        o_parts, lse_parts = o_parts.numpy(), lse_parts.numpy()
+        mx = lse_parts.max(axis=0)
+        w = np.where(np.isfinite(lse_parts), np.exp(lse_parts - mx), 0.0)
+        acc = (w[..., None] * np.nan_to_num(o_parts)).sum(axis=0)
+        tot = w.sum(axis=0)
+        return acc / tot[..., None], mx + np.log(tot)
+
+
+def test_shards_with_pairs():
+    """The ring computes only the shards holding an allowed pair for some row."""
+    for mask, window in (("none", 0), ("causal", 0), ("window", 5), ("window", 40),
+                         ("causal_window", 0), ("causal_window", 17), ("causal_window", 100)):
+        for r in range(4):
+            for s in range(4):
+                Ls = 16
+                rows = range(r * Ls, (r + 1) * Ls)
+                keys = range(s * Ls, (s + 1) * Ls)
+                brute = any(
+                    mask == "none" or (mask == "causal" and j <= i) or
+                    (mask == "window" and abs(i - j) <= window) or
+                    (mask == "causal_window" and j <= i and i - j <= window)
+                    for i in rows for j in keys)
+                assert seqpar.shard_has_pairs(r, s, Ls, mask, window) == brute, (mask, window, r, s)
 
 
 def _free_port():
@@ -68,7 +108,8 @@ def _rank_main(rank, world, port, q, k, v, mask, window, result):
 
 
 @pytest.mark.parametrize("world,mask,window", [(2, "causal", 0), (2, "none", 0),
-                                               (2, "window", 9), (3, "causal_window", 13)])
+                                               (2, "window", 9), (3, "causal_window", 13),
+                                               (3, "window", 30), (4, "causal", 0)])
 def test_gloo_ranks_return_their_rows_of_the_definition(world, mask, window):
     import oracle
 

@@ -19,6 +19,7 @@ import torch.distributed as dist
 
 import exact_blockwise_head_b200 as ebh
 from exact_blockwise_head_b200 import seqpar
+import oracle
 from tests import gpu_helpers as G
 
 pytestmark = pytest.mark.gpu
@@ -127,6 +128,63 @@ def test_emulated_ranks_give_the_definition(S, mask, window):
     one_o, one_l = G.gpu_forward(q, k, v, mask=mask, window=window)
     assert np.abs(out - one_o).max() <= G.BF16_OUT_ATOL
     assert np.abs(lse - one_l).max() <= G.BF16_LSE_ATOL
+
+
+@pytest.mark.parametrize("S,mask,window", [(4, "causal", 0), (2, "none", 0),
+                                           (4, "causal_window", 700), (3, "window", 250),
+                                           (3, "window", 600), (2, "causal_window", 0)])
+def test_emulated_ring_steps_give_the_definition(S, mask, window):
+    """The ring's steps run one rank after another: each rank's query rows
+    against every key shard that holds an allowed pair (attn_fwd_partial at
+    the signed offset (r - s) Ls, the shard read where it lies), then the
+    exact merge of those partials (attn_merge_rows at row offset r Ls)."""
+    B, H, Ls, d = 1, 2, 512, 128
+    L = S * Ls
+    q, k, v = G.rand_qkv(B, H, L, d, seed=S * 37 + window)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    outs, lses = [], []
+    for r in range(S):
+        qr = qd[:, :, r * Ls:(r + 1) * Ls].contiguous()
+        o_parts = torch.full((S, B, H, Ls, d), float("nan"), dtype=torch.float32, device="cuda")
+        l_parts = torch.full((S, B, H, Ls), float("nan"), dtype=torch.float32, device="cuda")
+        for s in range(S):
+            if seqpar.shard_has_pairs(r, s, Ls, mask, window):
+                ebh.forward_partial(qr, kd[:, :, s * Ls:(s + 1) * Ls].contiguous(),
+                                    vd[:, :, s * Ls:(s + 1) * Ls].contiguous(), (r - s) * Ls,
+                                    o_parts[s], l_parts[s], mask=mask, window=window)
+        o, l = ebh.merge_rows(o_parts, l_parts, [s * Ls for s in range(S)] + [L], L, r * Ls,
+                              mask=mask, window=window)
+        outs.append(o)
+        lses.append(l)
+    torch.cuda.synchronize()
+    assert ebh.device_status(0) == ebh.ATTN_OK
+    out = torch.cat(outs, dim=2).double().cpu().numpy()
+    lse = torch.cat(lses, dim=2).double().cpu().numpy()
+    ref_o, ref_l = G.oracle_full(q, k, v, mask=mask, window=window)
+    G.check_bf16(out, lse, ref_o, ref_l, f"{S} emulated ring ranks {mask} w={window}")
+
+
+def test_partial_rows_outside_the_shard_write_empty_partials():
+    """Rows whose tile reaches a shard but which have no allowed key in it get
+    O = 0 and LSE = -inf (the merge's mask rule never reads them)."""
+    B, H, Ls, d = 1, 1, 256, 64
+    q, k, v = G.rand_qkv(B, H, 2 * Ls, d, seed=3)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o = torch.full((B, H, Ls, d), float("nan"), dtype=torch.float32, device="cuda")
+    l = torch.full((B, H, Ls), float("nan"), dtype=torch.float32, device="cuda")
+    # rows 0..255 against the keys 256..511 with a +-100 window: rows >= 156
+    # reach the shard, rows < 156 of the reaching tiles have no key in it
+    ebh.forward_partial(qd[:, :, :Ls].contiguous(), kd[:, :, Ls:].contiguous(),
+                        vd[:, :, Ls:].contiguous(), -Ls, o, l, mask="window", window=100)
+    torch.cuda.synchronize()
+    lh, oh = l.cpu().numpy()[0, 0], o.cpu().numpy()[0, 0]
+    assert np.isneginf(lh[128:156]).all() and (oh[128:156] == 0).all()
+    assert np.isfinite(lh[156:]).all()
+    ref_o, ref_l = oracle.attention_partial(q.float().numpy(), k.float().numpy(),
+                                            v.float().numpy(), Ls, 2 * Ls, mask="window",
+                                            window=100)
+    assert np.abs(oh[156:] - ref_o[0, 0, 156:Ls]).max() <= G.BF16_OUT_ATOL
+    assert np.abs(lh[156:] - ref_l[0, 0, 156:Ls]).max() <= G.BF16_LSE_ATOL
 
 
 def _free_port():
