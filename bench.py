@@ -400,6 +400,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--only", default=None, choices=["layer", "backward"],
+                    help="run only the multi-head attention layer or the backward sweep "
+                         "(one JSON line; for profiling those kernels)")
     ap.add_argument("--parallel", default="heads", choices=["heads", "seq"],
                     help="heads: shard (batch, head) pairs, no collective (default); "
                          "seq: shard the sequence, ring over the K/V shards")
@@ -419,6 +422,15 @@ def main():
 
     if args.impl == "reference":
         return reference_arm(args, w, world, rank)
+    if args.only is not None:
+        import torch
+
+        torch.cuda.set_device(local_rank)
+        res = sweep_layer(ebh, torch, steps=args.steps) if args.only == "layer" else \
+            sweep_backward(ebh, torch, steps=args.steps)
+        assert ebh.device_status(local_rank) == ebh.ATTN_OK, "a kernel wait ran out"
+        print(json.dumps({"only": args.only, **res}), flush=True)
+        return 0
     if args.parallel == "seq":
         return seq_parallel_arm(args, w, world, rank, local_rank)
 
