@@ -152,7 +152,7 @@ class ClockSampler:
         0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.0005):
+    def __init__(self, device_index: int, period_s: float = 0.0):
         self.samples = []
         self.reasons = 0
         self.period = period_s
@@ -177,7 +177,7 @@ class ClockSampler:
                 self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
             except Exception:  # noqa: BLE001
                 pass
-            time.sleep(self.period)
+            time.sleep(self.period)  # 0: only yields; one NVML query is ~0.1-1 ms
 
     def __enter__(self):
         if self._nvml is not None:
@@ -281,6 +281,12 @@ def time_gpu(fn, steps, stream, flush=None):
     return [s.elapsed_time(e) for s, e in zip(starts, ends)]
 
 
+def median(xs):
+    ys = sorted(xs)
+    n = len(ys)
+    return ys[n // 2] if n % 2 else 0.5 * (ys[n // 2 - 1] + ys[n // 2])
+
+
 def sweep_other(ebh, torch, names, steps=5, warmup=3):
     """Kernel-only TFLOP/s of the other workloads (inputs drawn on the GPU)."""
     res = {}
@@ -304,9 +310,10 @@ def sweep_other(ebh, torch, names, steps=5, warmup=3):
             fn()
         small = 3 * q.numel() * 2 < 126e6
         ms = time_gpu(fn, steps, stream, flush=(lambda: flush_buf.zero_()) if small else None)
-        avg = sum(ms) / len(ms)
+        avg = median(ms)
         fl = algorithmic_flops(w)
-        res[name] = {"ms": round(avg, 4), "tflops": round(fl / avg / 1e9, 1),
+        res[name] = {"ms": round(avg, 4), "ms_mean": round(sum(ms) / len(ms), 4), "stat": "median",
+                     "tflops": round(fl / avg / 1e9, 1),
                      "tokens_per_s": round(w.B * w.L / avg * 1e3, 1),
                      "l2": "flushed between steps" if small else "inputs larger than L2"}
         if small:
@@ -325,7 +332,7 @@ def sweep_other(ebh, torch, names, steps=5, warmup=3):
     return res
 
 
-def sweep_layer(ebh, torch, B=4, L=2048, E=512, H=8, steps=10):
+def sweep_layer(ebh, torch, B=4, L=2048, E=512, H=8, steps=20):
     """The whole multi-head attention layer of the MHA page (qkv projection,
     head split, attention, merge, out projection), at the 8-head L=2048,
     E=512 configuration, L2 flushed between steps."""
@@ -346,9 +353,11 @@ def sweep_layer(ebh, torch, B=4, L=2048, E=512, H=8, steps=10):
         fn()
     torch.cuda.synchronize()
     ms = time_gpu(fn, steps, torch.cuda.current_stream(), flush=lambda: flush_buf.zero_())
-    avg = sum(ms) / len(ms)
+    avg = median(ms)
     flops = 8.0 * B * L * E * E + 4.0 * B * H * L * L * (E // H)
-    return {"ms": round(avg, 4), "tokens_per_s": round(B * L / avg * 1e3, 1),
+    return {"ms": round(avg, 4), "ms_mean": round(sum(ms) / len(ms), 4), "steps": len(ms),
+            "stat": "median",
+            "tokens_per_s": round(B * L / avg * 1e3, 1),
             "tflops": round(flops / avg / 1e9, 1),
             "config": f"B={B} L={L} E={E} H={H}, no mask, bf16",
             "l2": "flushed between steps",
@@ -375,11 +384,13 @@ def sweep_backward(ebh, torch, name="causal_bf16_L8192_d128", steps=3):
     fn()
     torch.cuda.synchronize()
     ms = time_gpu(fn, steps, torch.cuda.current_stream())
-    avg = sum(ms) / len(ms)
+    avg = median(ms)
     flops = 10.0 * w.d * w.B * w.H * allowed_pairs(w.L, w.mask, w.window)
     peaks, _ = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    return {"workload": name, "ms": round(avg, 3), "tflops": round(flops / avg / 1e9, 2),
+    return {"workload": name, "ms": round(avg, 3), "ms_mean": round(sum(ms) / len(ms), 3),
+            "stat": "median",
+            "tflops": round(flops / avg / 1e9, 2),
             "frac_of_measured_bf16": round(flops / avg / 1e9 / peak, 4),
             "flops": "10 d per allowed pair (S, dP, dV, dK, dQ); the dQ kernel recomputes S "
                      "and dP, so the tensor cores execute 14 d per pair",
@@ -426,8 +437,10 @@ def main():
         import torch
 
         torch.cuda.set_device(local_rank)
-        res = sweep_layer(ebh, torch, steps=args.steps) if args.only == "layer" else \
-            sweep_backward(ebh, torch, steps=args.steps)
+        with ClockSampler(local_rank) as only_clk:
+            res = sweep_layer(ebh, torch, steps=args.steps) if args.only == "layer" else \
+                sweep_backward(ebh, torch, steps=args.steps)
+        res["clocks"] = only_clk.summary()
         assert ebh.device_status(local_rank) == ebh.ATTN_OK, "a kernel wait ran out"
         print(json.dumps({"only": args.only, **res}), flush=True)
         return 0
@@ -605,11 +618,16 @@ def main():
                   if n != w.name]
         del bufs
         # side measurements: a failure is recorded in the line, not fatal to it
-        for key, fn in (("other_workloads_kernel_only", lambda: sweep_other(ebh, torch, others)),
-                        ("mha_layer", lambda: sweep_layer(ebh, torch)),
-                        ("backward", lambda: sweep_backward(ebh, torch))):
+        # the short layer and backward sweeps first: after the long forward
+        # workloads the power cap holds the SM clock lower for a while (each
+        # sweep records the clocks it ran at)
+        for key, fn in (("mha_layer", lambda: sweep_layer(ebh, torch)),
+                        ("backward", lambda: sweep_backward(ebh, torch)),
+                        ("other_workloads_kernel_only", lambda: sweep_other(ebh, torch, others))):
             try:
-                line[key] = fn()
+                with ClockSampler(local_rank) as sweep_clk:
+                    line[key] = fn()
+                line[key]["clocks"] = sweep_clk.summary()
             except Exception as e:  # noqa: BLE001
                 line[key] = {"error": f"{type(e).__name__}: {e}"[:300]}
                 torch.cuda.synchronize()

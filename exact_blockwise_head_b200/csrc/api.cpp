@@ -509,6 +509,7 @@ int attn_fwd_splitkv(const attn_params* p, int num_splits, void* workspace,
   m.window = a.window;
   m.kv_len = a.L;
   m.q_offset = 0;
+  m.dependent = true;  // the partial kernel just before it on the stream
   st = ebh::launch_merge(m, static_cast<cudaStream_t>(stream), &err);
   if (st == ATTN_ERR_CUDA) g_last_cuda_error = static_cast<int>(err);
   return st;

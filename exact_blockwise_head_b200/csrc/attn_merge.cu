@@ -26,6 +26,9 @@ constexpr int kMergeWarps = 8;
 
 template <int D>
 __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const MergeArgs m) {
+  // in a dependent launch: the partials' writer has completed from here on
+  // (a no-op otherwise)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int E = D / 32;  // columns per lane
   const long long row = static_cast<long long>(blockIdx.x) * kMergeWarps + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -112,14 +115,18 @@ int launch_merge(const MergeArgs& m, cudaStream_t stream, cudaError_t* err) {
   const long long rows = static_cast<long long>(m.BH) * m.L;
   const long long blocks = (rows + kMergeWarps - 1) / kMergeWarps;
   if (blocks > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  if (m.d == 128) {
-    attn_merge_kernel<128><<<static_cast<unsigned>(blocks), kMergeWarps * 32, 0, stream>>>(m);
-  } else if (m.d == 64) {
-    attn_merge_kernel<64><<<static_cast<unsigned>(blocks), kMergeWarps * 32, 0, stream>>>(m);
-  } else {
-    return ATTN_ERR_UNSUPPORTED;
-  }
-  *err = cudaGetLastError();
+  if (m.d != 128 && m.d != 64) return ATTN_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(kMergeWarps * 32);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = m.dependent ? 1 : 0;
+  *err = m.d == 128 ? cudaLaunchKernelEx(&cfg, attn_merge_kernel<128>, m)
+                    : cudaLaunchKernelEx(&cfg, attn_merge_kernel<64>, m);
   return *err == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

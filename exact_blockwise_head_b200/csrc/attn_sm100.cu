@@ -37,6 +37,7 @@
 
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "attn.h"
 #include "kernels.h"
@@ -504,6 +505,7 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
   auto bar = [&](int i) -> uint32_t { return smem_addr(&bars[i]); };
 
   if (threadIdx.x == 0) {
+    grid_launch_dependents();
     for (int t = 0; t < kNQ; ++t) {
       mbar_init(bar(C::kBarQFull + t), 1);
       mbar_init(bar(C::kBarQEmpty + t), 1);
@@ -536,6 +538,9 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const uint64_t limit = p.timeout_ns;
+  // in a dependent launch, the set-up above overlapped the previous kernel;
+  // its outputs (this kernel's inputs) are read only from here on
+  grid_dependency_wait();
 
   // Registers: the softmax warpgroups hold a 128-wide score row per thread;
   // the producer / MMA warpgroup needs few.  kSoftmaxRegs * 256 +
@@ -1152,6 +1157,24 @@ int sm_count(int device, cudaError_t* err) {
   return cache[device];
 }
 
+// Launch with or without the programmatic-dependent-launch attribute (the
+// kernel's own griddepcontrol instructions do the rest).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), int grid, int threads, int smem,
+                          cudaStream_t stream, bool dependent, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int D, int BN>
 int launch_t(const FwdArgs& a, cudaStream_t stream, cudaError_t* err) {
   using C = Cfg<D, BN>;
@@ -1243,8 +1266,8 @@ int launch_t(const FwdArgs& a, cudaStream_t stream, cudaError_t* err) {
   p.num_units = static_cast<int>(units);
   p.timeout_ns = a.timeout_ns;
   const int grid = p.num_units < nsm ? p.num_units : nsm;
-  kernel<<<grid, Lay::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, p);
-  *err = cudaGetLastError();
+  *err = launch_kernel(kernel, grid, Lay::kThreads, C::kSmemBytes, stream, a.dependent, tq, tk, tv,
+                       to, p);
   return *err == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

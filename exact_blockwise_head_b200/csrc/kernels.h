@@ -37,6 +37,10 @@ struct FwdArgs {
   int split_keys = 0;
   float* o_part = nullptr;
   float* lse_part = nullptr;
+  // Programmatic dependent launch: the kernel may start while the previous
+  // kernel on the stream finishes (its set-up overlaps that kernel's tail)
+  // and waits for it before its first global memory access.
+  bool dependent = false;
 };
 
 // Merge of split-KV partials: for every row, the splits whose key range
@@ -57,6 +61,9 @@ struct MergeArgs {
   // (0 and L for a plain split-KV merge)
   int kv_len = 0;
   int q_offset = 0;
+  // launched as a dependent of the partial kernel before it on the stream
+  // (programmatic dependent launch; the kernel waits for it first)
+  bool dependent = false;
 };
 
 // Each returns an ATTN_* status; on ATTN_ERR_CUDA *err holds the CUDA code.
@@ -111,7 +118,8 @@ size_t mha_workspace_bytes(int B, int L, int E);
 // fp32 accumulation, on the tensor cores; N and K multiples of 8.  Defined
 // with the attention kernels.
 int launch_linear_bf16(const void* x, const void* w, const void* bias, void* y, int M, int N, int K,
-                       uint64_t timeout_ns, cudaStream_t stream, cudaError_t* err);
+                       uint64_t timeout_ns, cudaStream_t stream, cudaError_t* err,
+                       bool dependent = false);
 // On failure *err holds the CUDA error and *proj the failing projection (1 the
 // qkv projection, 2 the output projection; 0 the attention).
 int launch_mha(const MhaArgs& a, void* workspace, cudaStream_t stream, cudaError_t* err,

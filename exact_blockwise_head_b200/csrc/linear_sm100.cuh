@@ -76,6 +76,7 @@ __global__ void __launch_bounds__(kLinThreads, 1)
   const int n_k = (p.K + kLinBK - 1) / kLinBK;  // a ragged K tail loads as zeros
 
   if (threadIdx.x == 0) {
+    grid_launch_dependents();
     for (int s = 0; s < kLinStages; ++s) {
       mbar_init(bar(C::kBarFull + s), 1);
       mbar_init(bar(C::kBarEmpty + s), 1);
@@ -97,6 +98,8 @@ __global__ void __launch_bounds__(kLinThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const uint64_t limit = p.timeout_ns;
+  // in a dependent launch, X (and anything else) is read only from here on
+  grid_dependency_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -249,7 +252,8 @@ bool make_map_2d(CUtensorMap* map, const void* base, int rows, int cols, int box
 
 template <int BN>
 int launch_linear_t(const void* x, const void* w, const void* bias, void* y, int M, int N, int K,
-                    int nsm, uint64_t timeout_ns, cudaStream_t stream, cudaError_t* err) {
+                    int nsm, uint64_t timeout_ns, cudaStream_t stream, cudaError_t* err,
+                    bool dependent) {
   using C = LinCfg<BN>;
   int device = 0;
   if ((*err = cudaGetDevice(&device)) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -286,15 +290,15 @@ int launch_linear_t(const void* x, const void* w, const void* bias, void* y, int
   p.num_tiles = static_cast<int>(tiles);
   p.timeout_ns = timeout_ns;
   const int grid = p.num_tiles < nsm ? p.num_tiles : nsm;
-  linear_sm100_kernel<BN><<<grid, kLinThreads, C::kSmemBytes, stream>>>(tx, tw, ty, p);
-  *err = cudaGetLastError();
+  *err = launch_kernel(linear_sm100_kernel<BN>, grid, kLinThreads, C::kSmemBytes, stream, dependent,
+                       tx, tw, ty, p);
   return *err == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 }  // namespace
 
 int launch_linear_bf16(const void* x, const void* w, const void* bias, void* y, int M, int N, int K,
-                       uint64_t timeout_ns, cudaStream_t stream, cudaError_t* err) {
+                       uint64_t timeout_ns, cudaStream_t stream, cudaError_t* err, bool dependent) {
   *err = cudaSuccess;
   // rows of 16-byte multiples (the tensor maps' stride rule); ragged tiles
   // load zeros past N and K and their stores are clipped at M and N
@@ -307,8 +311,8 @@ int launch_linear_bf16(const void* x, const void* w, const void* bias, void* y, 
   // at least two of them
   const long long tiles256 = static_cast<long long>((M + kLinBM - 1) / kLinBM) * ((N + 255) / 256);
   if (tiles256 >= 2LL * nsm)
-    return launch_linear_t<256>(x, w, bias, y, M, N, K, nsm, timeout_ns, stream, err);
-  return launch_linear_t<128>(x, w, bias, y, M, N, K, nsm, timeout_ns, stream, err);
+    return launch_linear_t<256>(x, w, bias, y, M, N, K, nsm, timeout_ns, stream, err, dependent);
+  return launch_linear_t<128>(x, w, bias, y, M, N, K, nsm, timeout_ns, stream, err, dependent);
 }
 
 }  // namespace ebh

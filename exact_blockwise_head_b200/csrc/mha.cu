@@ -65,6 +65,9 @@ int launch_mha(const MhaArgs& a, void* workspace, cudaStream_t stream, cudaError
   f.window = a.window;
   f.block_n = 128;
   f.timeout_ns = a.timeout_ns;
+  // the attention and the output projection start while the kernel before
+  // them drains, and wait for it before reading its output
+  f.dependent = true;
   const long long E3 = 3LL * a.E;
   for (int x = 0; x < 3; ++x) {
     f.stride[x][0] = E3;
@@ -76,7 +79,8 @@ int launch_mha(const MhaArgs& a, void* workspace, cudaStream_t stream, cudaError
   f.stride[3][2] = static_cast<long long>(a.E) * a.L;
   st = launch_fwd_bf16_sm100(f, stream, err);
   if (st != ATTN_OK) return st;
-  st = launch_linear_bf16(ctx, a.w_out, a.b_out, a.y, M, a.E, a.E, a.timeout_ns, stream, err);
+  st = launch_linear_bf16(ctx, a.w_out, a.b_out, a.y, M, a.E, a.E, a.timeout_ns, stream, err,
+                          /*dependent=*/true);
   if (st != ATTN_OK) *proj = 2;
   return st;
 }

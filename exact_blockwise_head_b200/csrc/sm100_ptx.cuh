@@ -90,6 +90,18 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// ---------------------------------------------------------------- grid dependency
+// Programmatic dependent launch: let the next kernel on the stream be
+// scheduled (its CTAs start once this grid's CTAs leave their SMs), and wait
+// until the previous kernel has completed and its writes are visible.  Both
+// are no-ops for a kernel launched without the dependent-launch attribute.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
