@@ -32,6 +32,11 @@
 // tcgen05 MMAs complete in issue order, "S_t(j) done" also means
 // "P_t(j-1).V done", which lets a softmax thread rescale its own rows of O_t
 // without any further barrier.
+// At d = 64 the columns leave room for P in its own block (S_0 | S_1 | P_0 |
+// P_1 | O_0 | O_1): S_t(j+1) is then issued as soon as the softmax group has
+// loaded S_t(j), one block ahead of P_t(j).V, the groups run without turns,
+// and a softmax thread waits for the previous P_t.V product before it writes
+// P_t or rescales O_t.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -166,12 +171,19 @@ struct Cfg {
   static constexpr int kBarOEmpty = kBarOFull + kNQ;       // [kNQ]
   static constexpr int kBarTok = kBarOEmpty + kNQ;        // [kNQ]
   static constexpr int kBarDrain = kBarTok + kNQ;
-  static constexpr int kNumBars = kBarDrain + 1;
+  // P in its own tensor-memory columns (d = 64, two-tile units): S_t(j+1)
+  // is issued as soon as the softmax has loaded S_t(j), one block ahead of
+  // P_t(j) V_j, and the two softmax groups run without turns
+  static constexpr bool kDecouple = D == 64 && kNQ == 2;
+  static constexpr int kBarSCons = kBarDrain + 1;     // [kNQ]: S_t loaded into registers
+  static constexpr int kBarPEmpty = kBarSCons + kNQ;  // [kNQ]: P_t's columns read by P.V
+  static constexpr int kNumBars = kBarPEmpty + kNQ;
   static constexpr int kSmemBytes = 1024 + kSmemQ + kSmemKV + kSmemO + 8 * kNumBars + 16;
-  static constexpr int kTmemNeed = kNQ * BN + kNQ * D;
+  static constexpr int kTmemNeed = kNQ * BN + (kDecouple ? kNQ * BN / 2 : 0) + kNQ * D;
   static constexpr int kTmemCols = kTmemNeed <= 256 ? 256 : 512;
-  static constexpr int kColS = 0;            // + t * BN
-  static constexpr int kColO = kNQ * BN;     // + t * D
+  static constexpr int kColS = 0;                                       // + t * BN
+  static constexpr int kColP = kDecouple ? kNQ * BN : 0;                // + t * BN / 2
+  static constexpr int kColO = kNQ * BN + (kDecouple ? kNQ * BN / 2 : 0);  // + t * D
   static_assert(kTmemNeed <= 512, "tensor memory budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
@@ -521,6 +533,12 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
       mbar_init(bar(C::kBarKVEmpty + s), 1);
     }
     mbar_init(bar(C::kBarDrain), 1);
+    if constexpr (C::kDecouple) {
+      for (int t = 0; t < kNQ; ++t) {
+        mbar_init(bar(C::kBarSCons + t), kSoftmaxThreads);
+        mbar_init(bar(C::kBarPEmpty + t), 1);
+      }
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -538,9 +556,6 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const uint64_t limit = p.timeout_ns;
-  // in a dependent launch, the set-up above overlapped the previous kernel;
-  // its outputs (this kernel's inputs) are read only from here on
-  grid_dependency_wait();
 
   // Registers: the softmax warpgroups hold a 128-wide score row per thread;
   // the producer / MMA warpgroup needs few.  kSoftmaxRegs * 256 +
@@ -555,6 +570,10 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
       // The whole warp walks the schedule (its counters stay warp-uniform);
       // one elected lane issues the copies.
       const bool leader = elect_one_sync();
+      // In a dependent launch the set-up above overlapped the previous
+      // kernel; its outputs are read from here on.  The other roles touch
+      // global memory only after data these loads brought in.
+      grid_dependency_wait();
       {
         int kv_it = 0;
         int q_cnt[kNQ] = {};
@@ -668,7 +687,8 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
         auto issue_pv = [&](int t, int vst, bool first) -> bool {
           const uint32_t b0 = lo_v + vst * kStageUnits;
           const uint32_t d = tmem + C::kColO + t * D;
-          const uint32_t a = tmem + C::kColS + t * BN;
+          const uint32_t a =
+              tmem + (C::kDecouple ? C::kColP + t * (BN / 2) : C::kColS + t * BN);
   #pragma unroll
           for (int h = 0; h < 2; ++h) {
             EBH_TRACE(kEvPWait + 10 * t, h);
@@ -692,6 +712,77 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
           return true;
         };
 
+        if constexpr (C::kDecouple) {
+          // S one block ahead: per step j, S_t(j+1) for both tiles (each as
+          // soon as its softmax group has loaded S_t(j)), then P_t(j) V_j
+          // for both.  Counters of S products issued and consumed run across
+          // units, like the barriers' phases.
+          uint32_t n_s0 = 0, n_s1 = 0;
+          for (int k = 0, u = unit_of(0, p); ok && u < p.num_units; u = unit_of(++k, p)) {
+            const TileWork w0 = decode_tile<BN>(u, 0, p);
+            const TileWork w1 = decode_tile<BN>(u, 1, p);
+            const int lo0 = w0.lo, hi0 = w0.valid ? w0.hi : w0.lo;
+            const int lo1 = w1.lo, hi1 = w1.valid ? w1.hi : w1.lo;
+            const bool has0 = hi0 > lo0, has1 = hi1 > lo1;
+            const int ulo = has0 ? (has1 ? min(lo0, lo1) : lo0) : (has1 ? lo1 : 0);
+            const int uhi = has0 ? (has1 ? max(hi0, hi1) : hi0) : (has1 ? hi1 : 0);
+            const int kv0 = kv_it;  // ring index of K_ulo; V_j follows K_j
+            kv_it += 2 * (uhi - ulo);
+            auto ring_wait = [&](int i) -> bool {
+              return warp_wait(bar(C::kBarKVFull + i % C::kStages), (i / C::kStages) & 1,
+                               abort_flag, limit);
+            };
+            // S_t(j) into S_t's columns once the previous S_t has been loaded
+            auto issue_s_ahead = [&](int t, int j, int kst) -> bool {
+              const uint32_t n = t ? n_s1 : n_s0;
+              if (n > 0 && !warp_wait(bar(C::kBarSCons + t), (n - 1) & 1, abort_flag, limit))
+                return false;
+              const int lo_t = t ? lo1 : lo0, hi_t = t ? hi1 : hi0;
+              if (j == lo_t &&
+                  !warp_wait(bar(C::kBarQFull + t), (par_q >> t) & 1, abort_flag, limit))
+                return false;
+              tc_fence_after();
+              issue_s(t, kst);
+              commit(bar(C::kBarSFull + t));
+              if (j == hi_t - 1) commit(bar(C::kBarQEmpty + t));
+              if (t)
+                ++n_s1;
+              else
+                ++n_s0;
+              return true;
+            };
+            auto s_step = [&](int j) -> bool {
+              const int ki = kv0 + 2 * (j - ulo);
+              if (!ring_wait(ki)) return false;
+              const int kst = ki % C::kStages;
+              if (j >= lo0 && j < hi0 && !issue_s_ahead(0, j, kst)) return false;
+              if (j >= lo1 && j < hi1 && !issue_s_ahead(1, j, kst)) return false;
+              commit(bar(C::kBarKVEmpty + kst));  // K_j no longer needed
+              return true;
+            };
+            if (uhi > ulo) ok = s_step(ulo);
+            for (int j = ulo; ok && j < uhi; ++j) {
+              if (j + 1 < uhi && !(ok = s_step(j + 1))) break;
+              const int vi = kv0 + 2 * (j - ulo) + 1;
+              if (!(ok = ring_wait(vi))) break;
+              const int vst = vi % C::kStages;
+              if (j >= lo0 && j < hi0) {
+                if (!(ok = issue_pv(0, vst, j == lo0))) break;
+                commit(bar(C::kBarPEmpty + 0));
+                if (j == hi0 - 1) commit(bar(C::kBarOFull + 0));
+              }
+              if (j >= lo1 && j < hi1) {
+                if (!(ok = issue_pv(1, vst, j == lo1))) break;
+                commit(bar(C::kBarPEmpty + 1));
+                if (j == hi1 - 1) commit(bar(C::kBarOFull + 1));
+              }
+              commit(bar(C::kBarKVEmpty + vst));  // V_j no longer needed
+            }
+            const uint32_t used = (has0 ? 1u : 0u) | (has1 ? 2u : 0u);
+            par_q ^= used;
+            par_oe ^= used;
+          }
+        } else
         for (int k = 0, u = unit_of(0, p); ok && u < p.num_units; u = unit_of(++k, p)) {
           // key-block ranges of the two Q tiles (empty range: tile absent)
           int lo0, hi0, lo1 = 0, hi1 = 0;  // a one-tile unit has no tile 1
@@ -789,6 +880,9 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(lbase) << 16;
     const uint32_t tS = tmem + lane_addr + C::kColS + t * BN;
     const uint32_t tO = tmem + lane_addr + C::kColO + t * D;
+    // P_t's bf16 pairs: over the first half of S_t, or in their own columns
+    const uint32_t tP = C::kDecouple ? tmem + lane_addr + C::kColP + t * (BN / 2) : tS;
+    uint32_t n_p = 0;  // P_t blocks written (own columns: P.V products awaited)
     const float cl2 = p.scale_log2;
     uint32_t phase = 0;  // bit 0: S_full parity, bit 1: O_full parity
     bool ok = true;
@@ -830,7 +924,7 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
         constexpr int kHalf = BN / 16;  // column groups of 8 per half
         uint32_t sr[BN / 2];
         tmem_ld_half<BN>(tS, sr);
-        {
+        if constexpr (!C::kDecouple) {
           const int jo = t == 0 ? j - 1 : j;  // the other tile's block that goes first
           if (jo >= o_lo && jo < o_hi) {
             const uint32_t kt = o_base + static_cast<uint32_t>(jo - o_lo);
@@ -842,6 +936,14 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
         }
         tmem_wait_ld();
         reg_fence_half<BN>(sr);
+        if constexpr (C::kDecouple) {
+          // P_t's columns and O_t are free once the previous P_t V product
+          // has completed
+          if (n_p > 0 &&
+              !(ok = warp_wait(bar(C::kBarPEmpty + t), (n_p - 1) & 1, abort_flag, limit)))
+            break;
+          ++n_p;
+        }
         tmem_ld_half<BN>(tS + BN / 2, sr + BN / 4);
         float* s = reinterpret_cast<float*>(sr);
         EBH_TRACE(kEvSLoaded, j);
@@ -865,13 +967,17 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
           const float l_a0 = l_a, l_b0 = l_b, lr_a0 = lr_a, lr_b0 = lr_b;
           EBH_TRACE(kEvMaxDone, j);
           if (full) {
-            probabilities<0, kHalf, kPolyOn>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
+            probabilities<0, kHalf, kPolyOn>(s, cl2, m_a, m_b, tP, l_a, l_b, lr_a, lr_b);
           } else {
-            probabilities<0, kHalf, false>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
+            probabilities<0, kHalf, false>(s, cl2, m_a, m_b, tP, l_a, l_b, lr_a, lr_b);
           }
           EBH_TRACE(kEvHalf1, j);
           tmem_wait_ld();
           reg_fence_half<BN>(sr + BN / 4);
+          if constexpr (C::kDecouple) {  // S_t's columns may take S_t(j+1)
+            tc_fence_before();
+            mbar_arrive(bar(C::kBarSCons + t));
+          }
           EBH_TRACE(kEvHalf2Loaded, j);
           if (!full) mask_groups<kHalf, 2 * kHalf>(s, t0, a_lo, a_hi, b_lo, b_hi);
           float mta, mtb;
@@ -895,7 +1001,7 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
             tc_fence_before();
             mbar_arrive(bar(C::kBarPFull + 2 * t));
             released_a = true;
-            store_p<kHalf, 2 * kHalf>(tS, pk2);
+            store_p<kHalf, 2 * kHalf>(tP, pk2);
           } else {
             // rare: redo the tile against the grown maximum
             float alpha_a = 1.f, alpha_b = 1.f;
@@ -912,7 +1018,7 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
             l_b = l_b0 * alpha_b;
             lr_b = lr_b0 * alpha_b;
             rescale_o_rows<D>(tO, alpha_a, alpha_b);
-            probabilities<0, 2 * kHalf, false>(s, cl2, m_a, m_b, tS, l_a, l_b, lr_a, lr_b);
+            probabilities<0, 2 * kHalf, false>(s, cl2, m_a, m_b, tP, l_a, l_b, lr_a, lr_b);
             EBH_TRACE(kEvHalf2, j);
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(C::kBarTok + t));
@@ -922,6 +1028,10 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
           // take the tile max as the reference before any exponential
           tmem_wait_ld();
           reg_fence_half<BN>(sr + BN / 4);
+          if constexpr (C::kDecouple) {
+            tc_fence_before();
+            mbar_arrive(bar(C::kBarSCons + t));
+          }
           if (!full) mask_groups<kHalf, 2 * kHalf>(s, t0, a_lo, a_hi, b_lo, b_hi);
           float mta, mtb;
           row_max_pair<BN>(s, mta, mtb);
@@ -954,7 +1064,7 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
           // a row with every key masked so far keeps m = -inf: subtract 0 so
           // that -inf - (-inf) never happens (its probabilities are all 0)
           probabilities<0, 2 * kHalf, false>(s, cl2, m_a == -INFINITY ? 0.f : m_a,
-                                      m_b == -INFINITY ? 0.f : m_b, tS, l_a, l_b, lr_a, lr_b);
+                                      m_b == -INFINITY ? 0.f : m_b, tP, l_a, l_b, lr_a, lr_b);
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(C::kBarTok + t));
         }

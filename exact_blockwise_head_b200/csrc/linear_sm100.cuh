@@ -98,8 +98,6 @@ __global__ void __launch_bounds__(kLinThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const uint64_t limit = p.timeout_ns;
-  // in a dependent launch, X (and anything else) is read only from here on
-  grid_dependency_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -108,6 +106,9 @@ __global__ void __launch_bounds__(kLinThreads, 1)
       tma_prefetch_desc(&tm_x);
       tma_prefetch_desc(&tm_w);
     }
+    // in a dependent launch, X is read from here on; the MMA and epilogue
+    // warps touch global memory only after data these loads brought in
+    grid_dependency_wait();
     int it = 0;  // K slices issued so far (ring position)
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
