@@ -277,6 +277,10 @@ def time_gpu(fn, steps, stream, flush=None):
         starts[i].record(stream)
         fn()
         ends[i].record(stream)
+    # poll rather than block: a blocking synchronize holds the interpreter
+    # lock, and the clock sampler's thread would take no sample meanwhile
+    while not ends[-1].query():
+        time.sleep(0.0002)
     torch.cuda.synchronize()
     return [s.elapsed_time(e) for s, e in zip(starts, ends)]
 
