@@ -368,6 +368,42 @@ def sweep_layer(ebh, torch, B=4, L=2048, E=512, H=8, steps=20):
             "flops": "8 B L E^2 (projections) + 4 B H L^2 d (attention)"}
 
 
+def sweep_splitkv(ebh, torch, steps=10):
+    """Split-KV on shapes with fewer 256-row work units than SMs (the case it
+    exists for): the plain forward against 2, 3 and 4 key runs, each with its
+    merge, L2 flushed between steps (kernel-only, inputs drawn on the GPU)."""
+    res = {}
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    for B, H, L, d, mask in ((1, 4, 8192, 128, "causal"), (1, 8, 4096, 128, "none")):
+        g = torch.Generator(device="cuda").manual_seed(7)
+        q, k, v = (torch.randn((B, H, L, d), device="cuda", generator=g).to(torch.bfloat16)
+                   for _ in range(3))
+        out = torch.empty_like(q)
+        lse = torch.empty((B, H, L), device="cuda", dtype=torch.float32)
+        fl = 4.0 * d * B * H * allowed_pairs(L, mask, 0)
+        entry = {"units": B * H * ((L + 255) // 256)}
+        for splits in (1, 2, 3, 4):
+            ws = torch.empty(ebh.splitkv_workspace_bytes(B, H, L, d, max(splits, 1)) + 256,
+                             dtype=torch.uint8, device="cuda")
+            if splits == 1:
+                fn = lambda: ebh.forward(q, k, v, mask=mask, out=out, lse=lse)  # noqa: E731
+            else:
+                fn = lambda: ebh.forward_splitkv(q, k, v, splits, mask=mask, out=out,  # noqa: E731
+                                                 lse=lse, workspace=ws)
+            for _ in range(3):
+                fn()
+            ms = median(time_gpu(fn, steps, stream, flush=lambda: flush_buf.zero_()))
+            entry["plain" if splits == 1 else f"splits_{splits}"] = {
+                "ms": round(ms, 4), "tflops": round(fl / ms / 1e9, 1)}
+            del ws
+        res[f"{mask}_bf16_B{B}_H{H}_L{L}_d{d}"] = entry
+        del q, k, v, out, lse
+    res["stat"] = "median"
+    res["l2"] = "flushed between steps"
+    return res
+
+
 def sweep_backward(ebh, torch, name="causal_bf16_L8192_d128", steps=3):
     """The backward (dQ, dK, dV by recomputation) on one workload.
     Algorithmic FLOPs: 10 d per allowed pair (the recomputed S, dP, and the
@@ -415,8 +451,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
-    ap.add_argument("--only", default=None, choices=["layer", "backward"],
-                    help="run only the multi-head attention layer or the backward sweep "
+    ap.add_argument("--only", default=None, choices=["layer", "backward", "splitkv"],
+                    help="run only the multi-head attention layer, the backward or the "
+                         "low-occupancy split-KV sweep "
                          "(one JSON line; for profiling those kernels)")
     ap.add_argument("--parallel", default="heads", choices=["heads", "seq"],
                     help="heads: shard (batch, head) pairs, no collective (default); "
@@ -442,8 +479,9 @@ def main():
 
         torch.cuda.set_device(local_rank)
         with ClockSampler(local_rank) as only_clk:
-            res = sweep_layer(ebh, torch, steps=args.steps) if args.only == "layer" else \
-                sweep_backward(ebh, torch, steps=args.steps)
+            only = {"layer": sweep_layer, "backward": sweep_backward,
+                    "splitkv": sweep_splitkv}[args.only]
+            res = only(ebh, torch, steps=args.steps)
         res["clocks"] = only_clk.summary()
         assert ebh.device_status(local_rank) == ebh.ATTN_OK, "a kernel wait ran out"
         print(json.dumps({"only": args.only, **res}), flush=True)
@@ -627,6 +665,7 @@ def main():
         # sweep records the clocks it ran at)
         for key, fn in (("mha_layer", lambda: sweep_layer(ebh, torch)),
                         ("backward", lambda: sweep_backward(ebh, torch)),
+                        ("splitkv_low_occupancy", lambda: sweep_splitkv(ebh, torch)),
                         ("other_workloads_kernel_only", lambda: sweep_other(ebh, torch, others))):
             try:
                 with ClockSampler(local_rank) as sweep_clk:

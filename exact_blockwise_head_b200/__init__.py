@@ -30,6 +30,8 @@ ATTN_ERR_CUDA = 4
 ATTN_ERR_TIMEOUT = 5
 ATTN_ERR_SCRATCH_LIMIT = 6
 NOALLOC_SCRATCH_BYTES = 32 << 20  # ATTN_NOALLOC_SCRATCH_BYTES
+ATTN_SPLITS_AUTO = 0  # num_splits: the library chooses (at most ATTN_SPLITS_AUTO_MAX runs)
+ATTN_SPLITS_AUTO_MAX = 2
 ATTN_DTYPE_BF16 = 0
 ATTN_DTYPE_F32 = 1
 
@@ -446,7 +448,9 @@ def splitkv_workspace_bytes(B, H, L, d, num_splits) -> int:
 def forward_splitkv(q, k, v, num_splits, scale=None, mask="none", window=0, block_n=0,
                     out=None, lse=None, want_lse=True, workspace=None, stream=None):
     """forward() with the key blocks cut into up to num_splits runs that run as
-    separate work units, then merged exactly.  bf16 only.  `workspace` is a
+    separate work units, then merged exactly (num_splits=ATTN_SPLITS_AUTO:
+    the library chooses; see attn_fwd_splitkv in include/attn.h).  bf16 only.
+    `workspace` is a
     CUDA uint8 tensor of at least splitkv_workspace_bytes(...) bytes (allocated
     here when omitted)."""
     import torch

@@ -129,7 +129,22 @@ int splitkv_check(const attn_params* p, int num_splits, int* runs, int* run_bloc
   int st = validate(p, &a);
   if (st != ATTN_OK) return st;
   if (p->dtype != ATTN_DTYPE_BF16) return ATTN_ERR_UNSUPPORTED;
-  if (num_splits < 1 || num_splits > kMaxSplits) return ATTN_ERR_INVALID;
+  if (num_splits < 0 || num_splits > kMaxSplits) return ATTN_ERR_INVALID;
+  if (num_splits == ATTN_SPLITS_AUTO) {
+    // A causal problem with no more 256-row work units than SMs runs one
+    // unit per SM, so its time is that of the longest unit (the last rows,
+    // which see every key): two key runs halve it.  Balanced masks and
+    // problems that fill the SMs gain nothing from the extra merge.
+    num_splits = 1;
+    if (a.mask_kind == kMaskCausal) {
+      int device = 0, nsm = 0;
+      if (cudaGetDevice(&device) != cudaSuccess ||
+          cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+      const long long units = static_cast<long long>(a.B) * a.H * ((a.L + 255) / 256);
+      if (units <= nsm) num_splits = 2;
+    }
+  }
   // whole key blocks per run; the last run may be shorter
   const int nkv = (a.L + a.block_n - 1) / a.block_n;
   *run_blocks = (nkv + num_splits - 1) / num_splits;
@@ -451,6 +466,7 @@ int attn_kv_tile_class(int L, int q_first, int q_last, int j, int mask_kind, int
 }
 
 size_t attn_splitkv_workspace_bytes(int B, int H, int L, int d, int num_splits) {
+  if (num_splits == ATTN_SPLITS_AUTO) num_splits = ATTN_SPLITS_AUTO_MAX;
   if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || num_splits < 1) return 0;
   const size_t rows = static_cast<size_t>(num_splits) * B * H * L;
   const size_t o_bytes = (rows * d * sizeof(float) + 255) / 256 * 256;

@@ -218,7 +218,8 @@ ATTN_API int attn_kv_full_range(int L, int q_first, int q_last, int mask_kind, i
 
 /*
  * Split-KV forward (bf16 path).  The key blocks are cut into up to
- * num_splits (1..64) contiguous runs; every (query tile, run) pair is an
+ * num_splits (1..64, or ATTN_SPLITS_AUTO below) contiguous runs; every
+ * (query tile, run) pair is an
  * independent work unit, which keeps all SMs busy when B*H*L/256 is small.
  * Each run writes an fp32 partial output normalised within the run and its
  * LSE into `workspace`, then attn_merge's rule combines the runs exactly
@@ -230,7 +231,18 @@ ATTN_API int attn_kv_full_range(int L, int q_first, int q_last, int mask_kind, i
  * always enough); it must not overlap any other argument.  Its contents on
  * entry do not matter.  With one run this is attn_fwd_ex and the workspace
  * is not touched.  Other arguments and errors as attn_fwd_ex.
+ *
+ * num_splits = ATTN_SPLITS_AUTO (0) lets the library choose: two runs for a
+ * causal mask when B*H*ceil(L/256) is at most the device's SM count (one
+ * work unit per SM, so the longest unit sets the time; measured on B200 at
+ * B=1 H=4 L=8192 d=128: 483 -> 692 TFLOP/s), one run otherwise (a balanced
+ * problem only pays for the merge).  attn_splitkv_workspace_bytes(..., 0)
+ * returns the size for ATTN_SPLITS_AUTO_MAX runs, enough for any choice.
+ * The choice reads the current device's SM count (ATTN_ERR_CUDA if that
+ * query fails).
  */
+#define ATTN_SPLITS_AUTO 0
+#define ATTN_SPLITS_AUTO_MAX 2
 ATTN_API size_t attn_splitkv_workspace_bytes(int B, int H, int L, int d, int num_splits);
 ATTN_API int attn_fwd_splitkv(const attn_params* p, int num_splits, void* workspace,
                               size_t workspace_bytes, void* stream);

@@ -163,8 +163,13 @@ def test_newer_entry_points_validate_before_any_device_work(lib):
     flat = (ctypes.c_int64 * 12)(*(good * 4))
     assert lib.attn_fwd_strided(ctypes.byref(pf), flat, None) == ebh.ATTN_ERR_UNSUPPORTED
     # split-KV: split count and workspace
-    assert lib.attn_fwd_splitkv(ctypes.byref(p), 0, None, 0, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_fwd_splitkv(ctypes.byref(p), -1, None, 0, None) == ebh.ATTN_ERR_INVALID
     assert lib.attn_fwd_splitkv(ctypes.byref(p), 65, None, 0, None) == ebh.ATTN_ERR_INVALID
+    # the automatic choice (0) takes at most two runs; its workspace query
+    # returns the size for two
+    assert ebh.ATTN_SPLITS_AUTO == 0
+    assert lib.attn_splitkv_workspace_bytes(2, 3, 1000, 128, 0) == \
+        lib.attn_splitkv_workspace_bytes(2, 3, 1000, 128, 2) > 0
     assert lib.attn_fwd_splitkv(ctypes.byref(p), 2, None, 0, None) == ebh.ATTN_ERR_INVALID
     # no-allocation split-KV: a problem whose partials exceed the scratch
     gb = 1 << 30  # tensors 1 GiB apart: the 64 MiB ones below do not overlap
@@ -184,7 +189,7 @@ def test_newer_entry_points_validate_before_any_device_work(lib):
     assert lib.attn_fwd_splitkv_noalloc(ctypes.byref(_params(B=1, H=32, L=8192, d=128,
                                                              block_n=96, **far)), 2,
                                         None) == ebh.ATTN_ERR_INVALID
-    assert lib.attn_fwd_splitkv_noalloc(ctypes.byref(big), 0, None) == ebh.ATTN_ERR_INVALID
+    assert lib.attn_fwd_splitkv_noalloc(ctypes.byref(big), -1, None) == ebh.ATTN_ERR_INVALID
     assert lib.attn_fwd_splitkv_noalloc(ctypes.byref(big), 65, None) == ebh.ATTN_ERR_INVALID
     assert lib.attn_fwd_splitkv_noalloc(None, 2, None) == ebh.ATTN_ERR_INVALID
     # backward: lse, gradients and workspace are required; block_n must be 0

@@ -55,6 +55,24 @@ def test_splitkv_matches_oracle(shape, mask, window, splits):
         G.check_bf16(out, lse, ref_o, ref_l, f"splitkv {shape} {mask} S={splits} bn={bn}")
 
 
+@pytest.mark.parametrize("shape,mask,expect_runs", [
+    ((1, 4, 2048, 128), "causal", 2),   # 32 work units: fewer than the SMs
+    ((2, 1, 900, 64), "none", 1),       # a balanced mask: never split
+    ((1, 2, 1000, 128), "window", 1),
+], ids=lambda c: str(c).replace(" ", ""))
+def test_splitkv_auto(shape, mask, expect_runs):
+    """num_splits=ATTN_SPLITS_AUTO matches the oracle and, bit for bit, the
+    explicit call with the run count the documented rule picks (the kernels
+    are deterministic)."""
+    q, k, v = G.rand_qkv(*shape, seed=sum(shape) + 11)
+    w = 200 if mask == "window" else 0
+    ref_o, ref_l = G.oracle_full(q, k, v, mask=mask, window=w)
+    out, lse = _splitkv(q, k, v, ebh.ATTN_SPLITS_AUTO, mask, w)
+    G.check_bf16(out, lse, ref_o, ref_l, f"splitkv auto {shape} {mask}")
+    out2, lse2 = _splitkv(q, k, v, expect_runs, mask, w)
+    assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
+
+
 def test_merge_of_oracle_partials():
     B, H, L, d = 1, 2, 900, 128
     q, k, v = G.rand_qkv(B, H, L, d, seed=77)
