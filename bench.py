@@ -375,7 +375,8 @@ def sweep_splitkv(ebh, torch, steps=10):
     res = {}
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
-    for B, H, L, d, mask in ((1, 4, 8192, 128, "causal"), (1, 8, 4096, 128, "none")):
+    for B, H, L, d, mask in ((1, 4, 8192, 128, "causal"), (1, 8, 4096, 128, "none"),
+                             (1, 1, 8192, 128, "causal"), (1, 2, 4096, 128, "none")):
         g = torch.Generator(device="cuda").manual_seed(7)
         q, k, v = (torch.randn((B, H, L, d), device="cuda", generator=g).to(torch.bfloat16)
                    for _ in range(3))
@@ -383,8 +384,8 @@ def sweep_splitkv(ebh, torch, steps=10):
         lse = torch.empty((B, H, L), device="cuda", dtype=torch.float32)
         fl = 4.0 * d * B * H * allowed_pairs(L, mask, 0)
         entry = {"units": B * H * ((L + 255) // 256)}
-        for splits in (1, 2, 3, 4):
-            ws = torch.empty(ebh.splitkv_workspace_bytes(B, H, L, d, max(splits, 1)) + 256,
+        for splits in (1, 2, 3, 4, 0):
+            ws = torch.empty(ebh.splitkv_workspace_bytes(B, H, L, d, splits) + 256,
                              dtype=torch.uint8, device="cuda")
             if splits == 1:
                 fn = lambda: ebh.forward(q, k, v, mask=mask, out=out, lse=lse)  # noqa: E731
@@ -394,7 +395,8 @@ def sweep_splitkv(ebh, torch, steps=10):
             for _ in range(3):
                 fn()
             ms = median(time_gpu(fn, steps, stream, flush=lambda: flush_buf.zero_()))
-            entry["plain" if splits == 1 else f"splits_{splits}"] = {
+            key = {1: "plain", 0: "auto"}.get(splits, f"splits_{splits}")
+            entry[key] = {
                 "ms": round(ms, 4), "tflops": round(fl / ms / 1e9, 1)}
             del ws
         res[f"{mask}_bf16_B{B}_H{H}_L{L}_d{d}"] = entry

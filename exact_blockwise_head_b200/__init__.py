@@ -31,7 +31,7 @@ ATTN_ERR_TIMEOUT = 5
 ATTN_ERR_SCRATCH_LIMIT = 6
 NOALLOC_SCRATCH_BYTES = 32 << 20  # ATTN_NOALLOC_SCRATCH_BYTES
 ATTN_SPLITS_AUTO = 0  # num_splits: the library chooses (at most ATTN_SPLITS_AUTO_MAX runs)
-ATTN_SPLITS_AUTO_MAX = 2
+ATTN_SPLITS_AUTO_MAX = 8
 ATTN_DTYPE_BF16 = 0
 ATTN_DTYPE_F32 = 1
 

@@ -124,6 +124,27 @@ int check_device_sm100() {
 namespace ebh {
 void set_last_cuda_error(cudaError_t e) { g_last_cuda_error = static_cast<int>(e); }
 
+// Key runs the automatic choice takes: enough (query tile, run) units to
+// cover the SMs once, at most ATTN_SPLITS_AUTO_MAX; with a causal mask at
+// least two whenever the units fit in one wave (one unit per SM: the longest
+// unit, the last rows, sets the time).  Balanced problems that already fill
+// the SMs keep one run: they would only pay for the merge.
+int auto_splits(long long units, bool causal, int nsm) {
+  long long s = units > 0 ? nsm / units : 1;
+  if (s < 1) s = 1;
+  if (s > ATTN_SPLITS_AUTO_MAX) s = ATTN_SPLITS_AUTO_MAX;
+  if (causal && units <= nsm && s < 2) s = 2;
+  return static_cast<int>(s);
+}
+
+int current_sm_count(int* nsm) {
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess ||
+      cudaDeviceGetAttribute(nsm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
 int splitkv_check(const attn_params* p, int num_splits, int* runs, int* run_blocks) {
   FwdArgs a;
   int st = validate(p, &a);
@@ -131,19 +152,10 @@ int splitkv_check(const attn_params* p, int num_splits, int* runs, int* run_bloc
   if (p->dtype != ATTN_DTYPE_BF16) return ATTN_ERR_UNSUPPORTED;
   if (num_splits < 0 || num_splits > kMaxSplits) return ATTN_ERR_INVALID;
   if (num_splits == ATTN_SPLITS_AUTO) {
-    // A causal problem with no more 256-row work units than SMs runs one
-    // unit per SM, so its time is that of the longest unit (the last rows,
-    // which see every key): two key runs halve it.  Balanced masks and
-    // problems that fill the SMs gain nothing from the extra merge.
-    num_splits = 1;
-    if (a.mask_kind == kMaskCausal) {
-      int device = 0, nsm = 0;
-      if (cudaGetDevice(&device) != cudaSuccess ||
-          cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
-        return ATTN_ERR_CUDA;
-      const long long units = static_cast<long long>(a.B) * a.H * ((a.L + 255) / 256);
-      if (units <= nsm) num_splits = 2;
-    }
+    int nsm = 0;
+    if ((st = current_sm_count(&nsm)) != ATTN_OK) return st;
+    const long long units = static_cast<long long>(a.B) * a.H * ((a.L + 255) / 256);
+    num_splits = auto_splits(units, a.mask_kind == kMaskCausal, nsm);
   }
   // whole key blocks per run; the last run may be shorter
   const int nkv = (a.L + a.block_n - 1) / a.block_n;
@@ -466,8 +478,16 @@ int attn_kv_tile_class(int L, int q_first, int q_last, int j, int mask_kind, int
 }
 
 size_t attn_splitkv_workspace_bytes(int B, int H, int L, int d, int num_splits) {
-  if (num_splits == ATTN_SPLITS_AUTO) num_splits = ATTN_SPLITS_AUTO_MAX;
-  if (B <= 0 || H <= 0 || L <= 0 || d <= 0 || num_splits < 1) return 0;
+  if (B <= 0 || H <= 0 || L <= 0 || d <= 0) return 0;
+  if (num_splits == ATTN_SPLITS_AUTO) {
+    // the current device's choice for a causal mask, which is never below
+    // that for any other mask; without a device, the most it could choose
+    int nsm = 0;
+    const long long units = static_cast<long long>(B) * H * ((L + 255) / 256);
+    num_splits = ebh::current_sm_count(&nsm) == ATTN_OK ? ebh::auto_splits(units, true, nsm)
+                                                        : ATTN_SPLITS_AUTO_MAX;
+  }
+  if (num_splits < 1) return 0;
   const size_t rows = static_cast<size_t>(num_splits) * B * H * L;
   const size_t o_bytes = (rows * d * sizeof(float) + 255) / 256 * 256;
   return o_bytes + rows * sizeof(float);

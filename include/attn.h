@@ -232,17 +232,22 @@ ATTN_API int attn_kv_full_range(int L, int q_first, int q_last, int mask_kind, i
  * entry do not matter.  With one run this is attn_fwd_ex and the workspace
  * is not touched.  Other arguments and errors as attn_fwd_ex.
  *
- * num_splits = ATTN_SPLITS_AUTO (0) lets the library choose: two runs for a
- * causal mask when B*H*ceil(L/256) is at most the device's SM count (one
- * work unit per SM, so the longest unit sets the time; measured on B200 at
- * B=1 H=4 L=8192 d=128: 483 -> 692 TFLOP/s), one run otherwise (a balanced
- * problem only pays for the merge).  attn_splitkv_workspace_bytes(..., 0)
- * returns the size for ATTN_SPLITS_AUTO_MAX runs, enough for any choice.
- * The choice reads the current device's SM count (ATTN_ERR_CUDA if that
- * query fails).
+ * num_splits = ATTN_SPLITS_AUTO (0) lets the library choose from the
+ * current device's SM count and the U = B*H*ceil(L/256) work units of one
+ * run: floor(SMs / U) runs, at most ATTN_SPLITS_AUTO_MAX and at least one,
+ * and at least two for a causal mask when U <= SMs (one unit per SM, so the
+ * longest unit sets the time).  Measured on B200 (d=128, L2 flushed):
+ * causal B=1 H=4 L=8192 (U=128) 453 -> 664-692 TFLOP/s with two runs; no
+ * mask B=1 H=8 L=4096 (U=128) stays at one run (818-866; every split is
+ * slower); U=32: four runs, causal B=1 H=1 L=8192 122 -> 305, no mask B=1
+ * H=2 L=4096 227 -> 430.  attn_splitkv_workspace_bytes(..., 0) returns the
+ * size for the current device's choice under a causal mask (never less than
+ * under any other mask), or for ATTN_SPLITS_AUTO_MAX runs when no device
+ * answers; query it on the device the call will run on.  The call reads the
+ * SM count (ATTN_ERR_CUDA if that query fails).
  */
 #define ATTN_SPLITS_AUTO 0
-#define ATTN_SPLITS_AUTO_MAX 2
+#define ATTN_SPLITS_AUTO_MAX 8
 ATTN_API size_t attn_splitkv_workspace_bytes(int B, int H, int L, int d, int num_splits);
 ATTN_API int attn_fwd_splitkv(const attn_params* p, int num_splits, void* workspace,
                               size_t workspace_bytes, void* stream);

@@ -55,15 +55,36 @@ def test_splitkv_matches_oracle(shape, mask, window, splits):
         G.check_bf16(out, lse, ref_o, ref_l, f"splitkv {shape} {mask} S={splits} bn={bn}")
 
 
-@pytest.mark.parametrize("shape,mask,expect_runs", [
-    ((1, 4, 2048, 128), "causal", 2),   # 32 work units: fewer than the SMs
-    ((2, 1, 900, 64), "none", 1),       # a balanced mask: never split
-    ((1, 2, 1000, 128), "window", 1),
+def _auto_runs(shape, mask):
+    """The documented rule: floor(SMs / U) runs for U = B H ceil(L/256) units,
+    between 1 and ATTN_SPLITS_AUTO_MAX, at least 2 for a causal mask when
+    U <= SMs; then no more runs than key blocks (128 keys each)."""
+    B, H, L, _ = shape
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    units = B * H * ((L + 255) // 256)
+    s = min(max(nsm // units, 1), ebh.ATTN_SPLITS_AUTO_MAX)
+    if mask == "causal" and units <= nsm:
+        s = max(s, 2)
+    nkv = (L + 127) // 128
+    per = -(-nkv // s)
+    return -(-nkv // per)
+
+
+@pytest.mark.parametrize("shape,mask", [
+    ((1, 4, 2048, 128), "causal"),   # 32 work units: four runs on 148 SMs
+    ((2, 1, 900, 64), "none"),       # 8 units: as many runs as key blocks
+    ((1, 2, 1000, 128), "window"),
+    ((1, 40, 1024, 64), "none"),     # 160 units fill the SMs: one run
+    ((1, 40, 1024, 64), "causal"),
 ], ids=lambda c: str(c).replace(" ", ""))
-def test_splitkv_auto(shape, mask, expect_runs):
+def test_splitkv_auto(shape, mask):
     """num_splits=ATTN_SPLITS_AUTO matches the oracle and, bit for bit, the
     explicit call with the run count the documented rule picks (the kernels
-    are deterministic)."""
+    are deterministic); its workspace query covers that count."""
+    expect_runs = _auto_runs(shape, mask)
+    B, H, L, d = shape
+    assert ebh.splitkv_workspace_bytes(B, H, L, d, 0) >= \
+        ebh.splitkv_workspace_bytes(B, H, L, d, expect_runs)
     q, k, v = G.rand_qkv(*shape, seed=sum(shape) + 11)
     w = 200 if mask == "window" else 0
     ref_o, ref_l = G.oracle_full(q, k, v, mask=mask, window=w)
