@@ -782,82 +782,84 @@ __global__ void __launch_bounds__(Layout<BN>::kThreads, 1)
             par_q ^= used;
             par_oe ^= used;
           }
-        } else
-        for (int k = 0, u = unit_of(0, p); ok && u < p.num_units; u = unit_of(++k, p)) {
-          // key-block ranges of the two Q tiles (empty range: tile absent)
-          int lo0, hi0, lo1 = 0, hi1 = 0;  // a one-tile unit has no tile 1
-          {
-            const TileWork w0 = decode_tile<BN>(u, 0, p);
-            lo0 = w0.lo; hi0 = w0.valid ? w0.hi : w0.lo;
-            if constexpr (kNQ == 2) {
-              const TileWork w1 = decode_tile<BN>(u, 1, p);
-              lo1 = w1.lo; hi1 = w1.valid ? w1.hi : w1.lo;
+        } else {
+          // d = 128, and one-tile units: P over S_t, the groups take turns
+          for (int k = 0, u = unit_of(0, p); ok && u < p.num_units; u = unit_of(++k, p)) {
+            // key-block ranges of the two Q tiles (empty range: tile absent)
+            int lo0, hi0, lo1 = 0, hi1 = 0;  // a one-tile unit has no tile 1
+            {
+              const TileWork w0 = decode_tile<BN>(u, 0, p);
+              lo0 = w0.lo; hi0 = w0.valid ? w0.hi : w0.lo;
+              if constexpr (kNQ == 2) {
+                const TileWork w1 = decode_tile<BN>(u, 1, p);
+                lo1 = w1.lo; hi1 = w1.valid ? w1.hi : w1.lo;
+              }
             }
+            const bool has0 = hi0 > lo0, has1 = hi1 > lo1;
+            const int ulo = has0 ? (has1 ? min(lo0, lo1) : lo0) : (has1 ? lo1 : 0);
+            const int uhi = has0 ? (has1 ? max(hi0, hi1) : hi0) : (has1 ? hi1 : 0);
+            int pend_v = -1;  // ring stage of V_(j-1) still owed a P_1 . V product
+            for (int j = ulo; ok && j < uhi; ++j) {
+              const int kst = kv_it % C::kStages;
+              const uint32_t kph = (kv_it / C::kStages) & 1;
+              const int vst = (kv_it + 1) % C::kStages;
+              const uint32_t vph = ((kv_it + 1) / C::kStages) & 1;
+              kv_it += 2;
+              EBH_TRACE(kEvKWait, j);
+              if (!(ok = warp_wait(bar(C::kBarKVFull + kst), kph, abort_flag, limit))) break;
+              EBH_TRACE(kEvKReady, j);
+              const bool in0 = j >= lo0 && j < hi0, in1 = j >= lo1 && j < hi1;
+              if (in0) {
+                if (j == lo0 && !(ok = warp_wait(bar(C::kBarQFull + 0), par_q & 1, abort_flag,
+                                                    limit)))
+                  break;
+                tc_fence_after();
+                issue_s(0, kst);
+                EBH_TRACE(kEvSIssued + 0, j);
+                commit(bar(C::kBarSFull + 0));
+                if (j == hi0 - 1) commit(bar(C::kBarQEmpty + 0));
+              }
+              if (pend_v >= 0) {
+                if (!(ok = issue_pv(1, pend_v, j - 1 == lo1))) break;
+                commit(bar(C::kBarKVEmpty + pend_v));
+                if (j - 1 == hi1 - 1) commit(bar(C::kBarOFull + 1));
+                pend_v = -1;
+              }
+              if (in1) {
+                if (j == lo1 && !(ok = warp_wait(bar(C::kBarQFull + 1), (par_q >> 1) & 1,
+                                                    abort_flag, limit)))
+                  break;
+                tc_fence_after();
+                issue_s(1, kst);
+                EBH_TRACE(kEvSIssued + 1, j);
+                commit(bar(C::kBarSFull + 1));
+                if (j == hi1 - 1) commit(bar(C::kBarQEmpty + 1));
+              }
+              commit(bar(C::kBarKVEmpty + kst));  // K_j no longer needed
+              EBH_TRACE(kEvVWait, j);
+              if (!(ok = warp_wait(bar(C::kBarKVFull + vst), vph, abort_flag, limit))) break;
+              EBH_TRACE(kEvVReady, j);
+              if (in0) {
+                if (!(ok = issue_pv(0, vst, j == lo0))) break;
+                if (j == hi0 - 1) commit(bar(C::kBarOFull + 0));
+              }
+              if (in1) {
+                pend_v = vst;
+              } else {
+                commit(bar(C::kBarKVEmpty + vst));
+              }
+            }
+            if (ok && pend_v >= 0) {
+              if ((ok = issue_pv(1, pend_v, uhi - 1 == lo1))) {
+                commit(bar(C::kBarKVEmpty + pend_v));
+                if (uhi - 1 == hi1 - 1) commit(bar(C::kBarOFull + 1));
+              }
+            }
+            // Q tiles and O accumulators used by this unit move to their next phase
+            const uint32_t used = (has0 ? 1u : 0u) | (has1 ? 2u : 0u);
+            par_q ^= used;
+            par_oe ^= used;
           }
-          const bool has0 = hi0 > lo0, has1 = hi1 > lo1;
-          const int ulo = has0 ? (has1 ? min(lo0, lo1) : lo0) : (has1 ? lo1 : 0);
-          const int uhi = has0 ? (has1 ? max(hi0, hi1) : hi0) : (has1 ? hi1 : 0);
-          int pend_v = -1;  // ring stage of V_(j-1) still owed a P_1 . V product
-          for (int j = ulo; ok && j < uhi; ++j) {
-            const int kst = kv_it % C::kStages;
-            const uint32_t kph = (kv_it / C::kStages) & 1;
-            const int vst = (kv_it + 1) % C::kStages;
-            const uint32_t vph = ((kv_it + 1) / C::kStages) & 1;
-            kv_it += 2;
-            EBH_TRACE(kEvKWait, j);
-            if (!(ok = warp_wait(bar(C::kBarKVFull + kst), kph, abort_flag, limit))) break;
-            EBH_TRACE(kEvKReady, j);
-            const bool in0 = j >= lo0 && j < hi0, in1 = j >= lo1 && j < hi1;
-            if (in0) {
-              if (j == lo0 && !(ok = warp_wait(bar(C::kBarQFull + 0), par_q & 1, abort_flag,
-                                                  limit)))
-                break;
-              tc_fence_after();
-              issue_s(0, kst);
-              EBH_TRACE(kEvSIssued + 0, j);
-              commit(bar(C::kBarSFull + 0));
-              if (j == hi0 - 1) commit(bar(C::kBarQEmpty + 0));
-            }
-            if (pend_v >= 0) {
-              if (!(ok = issue_pv(1, pend_v, j - 1 == lo1))) break;
-              commit(bar(C::kBarKVEmpty + pend_v));
-              if (j - 1 == hi1 - 1) commit(bar(C::kBarOFull + 1));
-              pend_v = -1;
-            }
-            if (in1) {
-              if (j == lo1 && !(ok = warp_wait(bar(C::kBarQFull + 1), (par_q >> 1) & 1,
-                                                  abort_flag, limit)))
-                break;
-              tc_fence_after();
-              issue_s(1, kst);
-              EBH_TRACE(kEvSIssued + 1, j);
-              commit(bar(C::kBarSFull + 1));
-              if (j == hi1 - 1) commit(bar(C::kBarQEmpty + 1));
-            }
-            commit(bar(C::kBarKVEmpty + kst));  // K_j no longer needed
-            EBH_TRACE(kEvVWait, j);
-            if (!(ok = warp_wait(bar(C::kBarKVFull + vst), vph, abort_flag, limit))) break;
-            EBH_TRACE(kEvVReady, j);
-            if (in0) {
-              if (!(ok = issue_pv(0, vst, j == lo0))) break;
-              if (j == hi0 - 1) commit(bar(C::kBarOFull + 0));
-            }
-            if (in1) {
-              pend_v = vst;
-            } else {
-              commit(bar(C::kBarKVEmpty + vst));
-            }
-          }
-          if (ok && pend_v >= 0) {
-            if ((ok = issue_pv(1, pend_v, uhi - 1 == lo1))) {
-              commit(bar(C::kBarKVEmpty + pend_v));
-              if (uhi - 1 == hi1 - 1) commit(bar(C::kBarOFull + 1));
-            }
-          }
-          // Q tiles and O accumulators used by this unit move to their next phase
-          const uint32_t used = (has0 ? 1u : 0u) | (has1 ? 2u : 0u);
-          par_q ^= used;
-          par_oe ^= used;
         }
         // No MMA may still be writing tensor memory when it is freed.
         commit(bar(C::kBarDrain));
