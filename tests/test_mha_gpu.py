@@ -78,3 +78,29 @@ def test_layer_rejects_bad_shapes():
     with pytest.raises(ebh.AttnError) as e:
         ebh.mha_forward(x, w, None, wo, None, num_heads=5)  # E % H != 0
     assert e.value.status == ebh.ATTN_ERR_INVALID
+
+
+def test_layer_back_to_back_dependent_launches():
+    """The layer's attention and output projection start while the kernel
+    before them drains (programmatic dependent launch) and wait for it before
+    reading its output.  Calls queued back to back on one stream, each on its
+    own inputs and sharing one workspace, must give bit for bit what each
+    call gives alone (the first layer of a call also follows the previous
+    call's output projection)."""
+    B, L, E, H = 2, 1024, 512, 8
+    calls = [_layer_inputs(B, L, E, seed=900 + i) for i in range(6)]
+    cuda = [[t.cuda() for t in c] for c in calls]
+    ws = torch.empty(ebh.mha_workspace_bytes(B, L, E) + 256, dtype=torch.uint8, device="cuda")
+    alone = []
+    for c in cuda:
+        y = torch.empty(B, L, E, dtype=torch.bfloat16, device="cuda")
+        ebh.mha_forward(*c, num_heads=H, mask="causal", y=y, workspace=ws)
+        torch.cuda.synchronize()
+        alone.append(y)
+    queued = [torch.empty(B, L, E, dtype=torch.bfloat16, device="cuda") for _ in cuda]
+    for c, y in zip(cuda, queued):
+        ebh.mha_forward(*c, num_heads=H, mask="causal", y=y, workspace=ws)
+    torch.cuda.synchronize()
+    assert ebh.device_status(0) == ebh.ATTN_OK
+    for i, (a, q) in enumerate(zip(alone, queued)):
+        assert torch.equal(a, q), f"call {i}: queued result differs from the call alone"

@@ -138,3 +138,25 @@ def test_full_mha_L2048_split_in_two():
     ref_o, ref_l = G.oracle_rows(q, k, v, bh_idx, row_idx, mask=w.mask, window=w.window)
     G.check_bf16(out.reshape(BH, w.L, w.d)[bh_idx, row_idx],
                  lse.reshape(BH, w.L)[bh_idx, row_idx], ref_o, ref_l, "C2 split 2")
+
+
+def test_splitkv_back_to_back_dependent_merge():
+    """The merge starts while the partial kernel before it drains and waits
+    for it before reading the partials.  Split-KV calls queued back to back
+    on one stream, on different inputs with one shared workspace, must give
+    bit for bit what each gives alone."""
+    shape = (1, 4, 2048, 128)
+    ins = [[t.cuda() for t in G.rand_qkv(*shape, seed=700 + i)] for i in range(5)]
+    B, H, L, d = shape
+    ws = torch.empty(ebh.splitkv_workspace_bytes(B, H, L, d, 4) + 256, dtype=torch.uint8,
+                     device="cuda")
+    alone = []
+    for q, k, v in ins:
+        o, l = ebh.forward_splitkv(q, k, v, 4, mask="causal", workspace=ws)
+        torch.cuda.synchronize()
+        alone.append((o, l))
+    queued = [ebh.forward_splitkv(q, k, v, 4, mask="causal", workspace=ws) for q, k, v in ins]
+    torch.cuda.synchronize()
+    assert ebh.device_status(0) == ebh.ATTN_OK
+    for i, ((a_o, a_l), (q_o, q_l)) in enumerate(zip(alone, queued)):
+        assert torch.equal(a_o, q_o) and torch.equal(a_l, q_l), f"call {i} differs"
