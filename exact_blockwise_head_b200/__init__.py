@@ -42,7 +42,7 @@ EXPORTED = ("attn_fwd", "attn_fwd_f32", "attn_fwd_ex", "attn_strerror", "attn_la
             "attn_fwd_splitkv", "attn_merge", "attn_abi_version", "attn_fwd_splitkv_noalloc",
             "attn_fwd_rows", "attn_seq_unshard", "attn_mha_workspace_bytes", "attn_mha_fwd",
             "attn_bwd_workspace_bytes", "attn_bwd", "attn_query_rows_for_keys",
-            "attn_fwd_strided", "attn_fwd_partial", "attn_merge_rows")
+            "attn_fwd_strided", "attn_fwd_partial", "attn_merge_rows", "attn_splitkv_auto_runs")
 
 
 class AttnParams(ctypes.Structure):

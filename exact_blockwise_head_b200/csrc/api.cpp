@@ -154,8 +154,7 @@ int splitkv_check(const attn_params* p, int num_splits, int* runs, int* run_bloc
   if (num_splits == ATTN_SPLITS_AUTO) {
     int nsm = 0;
     if ((st = current_sm_count(&nsm)) != ATTN_OK) return st;
-    const long long units = static_cast<long long>(a.B) * a.H * ((a.L + 255) / 256);
-    num_splits = auto_splits(units, a.mask_kind == kMaskCausal, nsm);
+    num_splits = attn_splitkv_auto_runs(a.B, a.H, a.L, a.mask_kind, nsm);
   }
   // whole key blocks per run; the last run may be shorter
   const int nkv = (a.L + a.block_n - 1) / a.block_n;
@@ -477,15 +476,23 @@ int attn_kv_tile_class(int L, int q_first, int q_last, int j, int mask_kind, int
   return ebh::kv_tile_class(L, q_first, q_last, j, mask_kind, window, block_n);
 }
 
+int attn_splitkv_auto_runs(int B, int H, int L, int mask_kind, int num_sms) {
+  if (B < 1 || H < 1 || L < 1 || num_sms < 1 || mask_kind < ATTN_MASK_NONE ||
+      mask_kind > ATTN_MASK_CAUSAL_WINDOW)
+    return 0;
+  const long long units = static_cast<long long>(B) * H * ((static_cast<long long>(L) + 255) / 256);
+  return ebh::auto_splits(units, mask_kind == ATTN_MASK_CAUSAL, num_sms);
+}
+
 size_t attn_splitkv_workspace_bytes(int B, int H, int L, int d, int num_splits) {
   if (B <= 0 || H <= 0 || L <= 0 || d <= 0) return 0;
   if (num_splits == ATTN_SPLITS_AUTO) {
     // the current device's choice for a causal mask, which is never below
     // that for any other mask; without a device, the most it could choose
     int nsm = 0;
-    const long long units = static_cast<long long>(B) * H * ((L + 255) / 256);
-    num_splits = ebh::current_sm_count(&nsm) == ATTN_OK ? ebh::auto_splits(units, true, nsm)
-                                                        : ATTN_SPLITS_AUTO_MAX;
+    num_splits = ebh::current_sm_count(&nsm) == ATTN_OK
+                     ? attn_splitkv_auto_runs(B, H, L, ATTN_MASK_CAUSAL, nsm)
+                     : ATTN_SPLITS_AUTO_MAX;
   }
   if (num_splits < 1) return 0;
   const size_t rows = static_cast<size_t>(num_splits) * B * H * L;

@@ -248,6 +248,12 @@ ATTN_API int attn_kv_full_range(int L, int q_first, int q_last, int mask_kind, i
  */
 #define ATTN_SPLITS_AUTO 0
 #define ATTN_SPLITS_AUTO_MAX 8
+/* The automatic choice as a pure host function (no device call): the number
+ * of key runs ATTN_SPLITS_AUTO takes for B, H, L and mask_kind (ATTN_MASK_*)
+ * on a device with num_sms SMs, before the cut to whole key blocks (the call
+ * never uses more runs than the problem has key blocks).  0 for arguments
+ * outside B, H, L, num_sms >= 1 or an unknown mask_kind. */
+ATTN_API int attn_splitkv_auto_runs(int B, int H, int L, int mask_kind, int num_sms);
 ATTN_API size_t attn_splitkv_workspace_bytes(int B, int H, int L, int d, int num_splits);
 ATTN_API int attn_fwd_splitkv(const attn_params* p, int num_splits, void* workspace,
                               size_t workspace_bytes, void* stream);

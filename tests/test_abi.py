@@ -166,8 +166,25 @@ def test_newer_entry_points_validate_before_any_device_work(lib):
     # split-KV: split count and workspace
     assert lib.attn_fwd_splitkv(ctypes.byref(p), -1, None, 0, None) == ebh.ATTN_ERR_INVALID
     assert lib.attn_fwd_splitkv(ctypes.byref(p), 65, None, 0, None) == ebh.ATTN_ERR_INVALID
-    # the automatic choice (0): without a device its workspace query answers
-    # for the most runs it could take
+    # the automatic choice, by hand on a 148-SM device: floor(SMs / units)
+    # runs in 1..8, at least 2 for a causal mask when the units fit in one wave
+    auto = lib.attn_splitkv_auto_runs
+    C, N, W, CW = (ebh.MASK_KINDS[m] for m in ("causal", "none", "window", "causal_window"))
+    assert auto(1, 4, 8192, C, 148) == 2      # 128 units: one wave, causal
+    assert auto(1, 8, 4096, N, 148) == 1      # 128 units, balanced
+    assert auto(1, 1, 8192, C, 148) == 4      # 32 units
+    assert auto(1, 2, 4096, N, 148) == 4
+    assert auto(1, 1, 256, W, 148) == 8       # 1 unit: capped at 8
+    assert auto(4, 8, 2048, N, 148) == 1      # 256 units fill the SMs
+    assert auto(4, 8, 2048, C, 148) == 1      # ... causal too: more than one wave
+    assert auto(1, 1, 8192, CW, 148) == 4     # the causal floor is for mask kind 1 only
+    assert auto(1, 37, 256, C, 37) == 2       # units == SMs: still one wave
+    assert auto(1, 1, 257, N, 148) == 8       # 2 units: 74 capped at 8
+    for bad in ((0, 1, 1, N, 148), (1, 0, 1, N, 148), (1, 1, 0, N, 148), (1, 1, 1, 4, 148),
+                (1, 1, 1, -1, 148), (1, 1, 1, N, 0)):
+        assert auto(*bad) == 0, bad
+    # without a device the workspace query answers for the most runs the
+    # automatic choice could take
     assert ebh.ATTN_SPLITS_AUTO == 0
     if not torch.cuda.is_available():
         assert lib.attn_splitkv_workspace_bytes(2, 3, 1000, 128, 0) == \
