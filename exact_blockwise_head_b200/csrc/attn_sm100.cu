@@ -96,8 +96,11 @@ constexpr int kPolyEvery = EBH_POLY_EVERY > 0 ? EBH_POLY_EVERY : 1;
 constexpr bool kPolyOn = EBH_POLY_EVERY > 0;
 constexpr bool kScalarMath = EBH_SCALAR_MATH != 0;
 // Lazy rescale: keep the stale max until the row max exceeds it by more than
-// 2^8 (probabilities then stay <= 256, far inside fp32/bf16 range).
-constexpr float kRescaleThreshold = 8.0f;
+// 16 (log2 units).  Probabilities then stay <= 2^16: bf16 and fp32 keep the
+// same relative precision at any magnitude, and even 2^16 times 2^17 keys
+// stays far below fp32 overflow.  Rows whose max keeps growing (peaked
+// scores) redo fewer blocks than with a threshold of 8.
+constexpr float kRescaleThreshold = 16.0f;
 
 // Pipeline trace for profiling builds (-DEBH_PIPELINE_TRACE): lane 0 of each
 // warp of CTA 0 appends (event << 56 | key block << 40 | clock64) records to
