@@ -96,11 +96,12 @@ constexpr int kPolyEvery = EBH_POLY_EVERY > 0 ? EBH_POLY_EVERY : 1;
 constexpr bool kPolyOn = EBH_POLY_EVERY > 0;
 constexpr bool kScalarMath = EBH_SCALAR_MATH != 0;
 // Lazy rescale: keep the stale max until the row max exceeds it by more than
-// 16 (log2 units).  Probabilities then stay <= 2^16: bf16 and fp32 keep the
-// same relative precision at any magnitude, and even 2^16 times 2^17 keys
-// stays far below fp32 overflow.  Rows whose max keeps growing (peaked
-// scores) redo fewer blocks than with a threshold of 8.
-constexpr float kRescaleThreshold = 16.0f;
+// 32 (log2 units).  Probabilities then stay <= 2^32: bf16 and fp32 keep the
+// same relative precision at any magnitude, and 2^32 times 2^30 keys times a
+// value's magnitude stays far below fp32 overflow (3.4e38).  Rows whose max
+// keeps growing (peaked scores) then almost never redo a block; a larger
+// jump still takes the exact redo path.
+constexpr float kRescaleThreshold = 32.0f;
 
 // Pipeline trace for profiling builds (-DEBH_PIPELINE_TRACE): lane 0 of each
 // warp of CTA 0 appends (event << 56 | key block << 40 | clock64) records to
