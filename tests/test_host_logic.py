@@ -139,3 +139,30 @@ def test_weak_scaling_gives_every_rank_the_same_size():
     for world in (1, 2, 4, 8):
         sizes = {b - a for a, b in (weak_scaling_heads(32, world, r) for r in range(world))}
         assert sizes == {32}
+
+
+def test_reference_arm_line_keeps_the_contract():
+    """`bench.py --impl reference` (the fp64 oracle on the host cores) prints
+    one JSON line with the bench contract's keys: the same metric, unit and
+    config as our arm, impl "reference", a cpu_baseline describing the run
+    and an e2e block with no host-device copies."""
+    import json
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                        "--warmup", "3", "--cpu-seconds", "1"], cwd=root, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC
+    assert line["unit"] == "TFLOP/s" and line["higher_is_better"] is True
+    assert line["value"] > 0 and line["steps"] == 1 and line["warmup"] == 3
+    assert line["config"]["workload"] == bench.DEFAULT_WORKLOAD
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
